@@ -1,0 +1,294 @@
+"""Pins of the fp64 oracle to facts outside itself (CPU only).
+
+Each test ties one oracle function to something the pages print, a closed form, an
+invariant, a library routine for a special case, or brute force on tiny inputs.  The
+``test_planted_*`` tests mutate a copy of an oracle function with a plausible mistake
+and check that the matching pin catches it.
+"""
+import inspect
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.dsa_oracle as O
+from synth import make_prefill, make_decode, WORKLOADS, PrefillSpec, DecodeSpec
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "pages_numbers.json")))
+SCALE = 1.0 / math.sqrt(576)
+
+
+# ----------------------------------------------------------------------------- number formats
+
+
+def test_bf16_decoder_all_patterns_match_library():
+    bits = np.arange(1 << 16, dtype=np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    got = O.bf16_to_f64(bits)
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    assert same.all()
+    assert O.bf16_to_f64(np.array([0x3F80, 0xC000, 0x0001]))[2] == 2.0 ** -133
+
+
+def test_e4m3_decoder_all_codes_match_library_and_hand_values():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = O.e4m3_to_f64(codes)
+    assert (((got == ref) | (np.isnan(got) & np.isnan(ref)))).all()
+    hand = O.e4m3_to_f64(np.array([0x7E, 0x01, 0x38, 0x08, 0xB8], dtype=np.uint8))
+    assert list(hand) == [448.0, 2.0 ** -9, 1.0, 2.0 ** -6, -1.0]
+
+
+def test_e4m3_encoder_matches_library_in_range():
+    rng = np.random.default_rng(7)
+    v = np.concatenate([rng.normal(0, 100, 20000), rng.normal(0, 1e-2, 5000),
+                        np.ldexp(1.0, np.arange(-12, 9))]).astype(np.float32)
+    v = np.clip(v, -448, 448).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert (O._encode_e4m3_rne_sat(v) == ref).all()
+
+
+def test_e4m3_encoder_ties_to_even_and_saturation():
+    enc = O._encode_e4m3_rne_sat
+    # 1.0625 lies halfway between 1.0 (m=0) and 1.125 (m=1): even -> 1.0
+    # 1.1875 lies halfway between 1.125 (m=1) and 1.25 (m=2): even -> 1.25
+    # subnormal step 2^-9: 0.5 step ties to 0, 1.5 steps ties to 2, 0.75 step rounds to 1
+    v = np.array([1.0625, 1.1875, 500.0, -1e9, 2.0 ** -10, 3 * 2.0 ** -10, 3 * 2.0 ** -11],
+                 dtype=np.float32)
+    assert list(enc(v)) == [0x38, 0x3A, 0x7E, 0xFE, 0x00, 0x02, 0x01]
+
+
+def test_quantize_rows_scale_rule():
+    x = np.array([[0.0] * 127 + [2.0], [0.0] * 128, [-3.0] + [1.5] * 127], dtype=np.float32)
+    from synth.generators import bf16_bits_np
+    codes, scale = O.quantize_e4m3_rows(bf16_bits_np(x), 128)
+    assert scale[0] == np.float32(2.0) / np.float32(448.0)
+    assert scale[1] == 1.0 and (codes[1] == 0).all()
+    assert codes[0, 127] == 0x7E and codes[2, 0] == 0xFE     # amax element maps to +-448
+    back = O.e4m3_to_f64(codes[2]) * scale[2]
+    assert abs(back[0] + 3.0) < 1e-6 and np.all(np.abs(back[1:] - 1.5) <= 1.5 * 2 ** -4)
+
+
+# ----------------------------------------------------------------------------- indexer
+
+
+def _unit_case():
+    """q[t,h] = a_h e_{i_h}, k[s] = e_s: x[t,h,s] = a_h [i_h == s], closed form below."""
+    H, D, N = 32, 128, 16
+    rng = np.random.default_rng(3)
+    a = rng.normal(size=(2, H))
+    ih = rng.integers(0, N, size=(2, H))
+    q = np.zeros((2, H, D))
+    for t in range(2):
+        for h in range(H):
+            q[t, h, ih[t, h]] = a[t, h]
+    k = np.eye(N, D)
+    w = rng.normal(size=(2, H))
+    expect = np.zeros((2, N))
+    for t in range(2):
+        for h in range(H):
+            expect[t, ih[t, h]] += w[t, h] * max(a[t, h], 0.0)
+    return q, w, k, expect
+
+
+def test_indexer_closed_form_unit_vectors(fn=None):
+    fn = fn or O.indexer_scores
+    q, w, k, expect = _unit_case()
+    got = fn(q, w, k, [16, 9])
+    assert np.allclose(got[0], expect[0], rtol=0, atol=1e-12)
+    assert np.allclose(got[1, :9], expect[1, :9], rtol=0, atol=1e-12)
+    assert np.all(np.isneginf(got[1, 9:]))
+
+
+def test_indexer_invariants():
+    rng = np.random.default_rng(5)
+    q, w, k = rng.normal(size=(3, 32, 128)), rng.normal(size=(3, 32)), rng.normal(size=(40, 128))
+    I = O.indexer_scores(q, w, k, [40] * 3)
+    assert np.allclose(O.indexer_scores(q, w, 2.5 * k, [40] * 3), 2.5 * I)       # positive homogeneity
+    assert np.allclose(O.indexer_scores(q, -w, k, [40] * 3), -I)                 # linear in w
+    qp, kn = np.abs(q), -np.abs(k)            # every dot product <= 0: ReLU zeroes all heads
+    assert (O.indexer_scores(qp, w, kn, [40] * 3) == 0).all()
+
+
+# ----------------------------------------------------------------------------- top-k
+
+
+def _rank_select(s, n, k):
+    """Brute force: position i is kept iff fewer than k entries beat it (larger, or equal and earlier)."""
+    keep = []
+    for i in range(n):
+        beat = sum(1 for j in range(n) if s[j] > s[i] or (s[j] == s[i] and j < i))
+        if beat < k:
+            keep.append(i)
+    return set(keep)
+
+
+def test_topk_brute_force_tiny(fn=None):
+    fn = fn or O.topk_row
+    rng = np.random.default_rng(11)
+    for trial in range(300):
+        n = int(rng.integers(1, 12))
+        k = int(rng.integers(1, 8))
+        s = rng.integers(-3, 4, size=n).astype(float)        # many ties
+        got = fn(s, n, k)
+        assert set(int(i) for i in got if i >= 0) == _rank_select(s, n, k)
+        assert (got[min(k, n):] == -1).all()
+
+
+def test_topk_exhaustive_sets_equal_best_sum():
+    s = np.array([0.3, -1.0, 2.0, 0.3, 5.0, -0.2, 0.0])
+    for k in range(1, 8):
+        best = max(itertools.combinations(range(7), k), key=lambda c: (sum(s[list(c)]), [-i for i in c]))
+        assert set(O.topk_row(s, 7, k)) == set(best)
+
+
+# ----------------------------------------------------------------------------- attention
+
+
+def _rand_qkv(L, seed=0):
+    rng = np.random.default_rng(seed)
+    return rng.normal(size=(64, 576)), rng.normal(size=(L, 576))
+
+
+def test_sparse_equals_dense_when_k_covers_history(fn=None):
+    fn = fn or O.sparse_mla_row
+    Q, KV = _rand_qkv(37)
+    for t in (0, 5, 36):
+        idx = O.topk_row(np.random.default_rng(t).normal(size=t + 1), t + 1, 64)
+        o1, l1 = fn(Q, KV, idx, SCALE)
+        o2, l2 = O.dense_causal_attention_row(Q, KV[:t + 1], SCALE)
+        assert np.allclose(o1, o2, rtol=1e-12, atol=1e-12) and np.allclose(l1, l2, rtol=1e-12)
+
+
+def test_first_row_is_its_own_value():
+    Q, KV = _rand_qkv(4)
+    o, lse = O.sparse_mla_row(Q, KV, np.array([0, -1, -1]), SCALE)
+    assert np.array_equal(o, np.broadcast_to(KV[0, :512], (64, 512)))
+    assert np.allclose(lse, SCALE * Q @ KV[0])
+
+
+def test_attention_weights_sum_to_one_and_order_free():
+    Q, KV = _rand_qkv(50, 1)
+    KV2 = KV.copy()
+    KV2[:, :512] = 0.75
+    idx = np.array([3, 17, 40, 2, -1, 9])
+    o, _ = O.sparse_mla_row(Q, KV2, idx, SCALE)
+    assert np.allclose(o, 0.75, atol=1e-14)
+    o1, l1 = O.sparse_mla_row(Q, KV, idx, SCALE)
+    o2, l2 = O.sparse_mla_row(Q, KV, idx[::-1], SCALE)
+    assert np.allclose(o1, o2, atol=1e-13) and np.allclose(l1, l2)
+
+
+def test_empty_selection():
+    Q, KV = _rand_qkv(3)
+    o, l = O.sparse_mla_row(Q, KV, np.array([-1, -1]), SCALE)
+    assert (o == 0).all() and np.isneginf(l).all()
+
+
+# ----------------------------------------------------------------------------- group / MTP / schedule
+
+
+def test_group_shared_layers_reuse_full_indices_exactly():
+    spec = PrefillSpec("t", L=48, k=8, n_layers=4, seed=9)
+    inp = make_prefill(spec)
+    rows = [0, 3, 7, 20, 47]
+    g = O.group_prefill(inp, rows)
+    for t in rows:
+        assert len([i for i in g["idx"][t] if i >= 0]) == min(8, t + 1)
+        for l in range(4):       # every layer equals attention with the Full layer's indices
+            o, ls = O.sparse_mla_row(O.bf16_to_f64(inp["Q"][l][t]), O.bf16_to_f64(inp["KV"][l]),
+                                     g["idx"][t], inp["softmax_scale"])
+            assert np.array_equal(o, g["O"][l][t])
+    # rows with t + 1 <= k select the whole causal history: dense attention
+    o, _ = O.dense_causal_attention_row(O.bf16_to_f64(inp["Q"][2][3]), O.bf16_to_f64(inp["KV"][2][:4]),
+                                        inp["softmax_scale"])
+    assert np.allclose(o, g["O"][2][3], atol=1e-12)
+
+
+def test_decode_mtp_rows_share_row0_indices():
+    spec = DecodeSpec("t", batch=2, ctx_lo=70, ctx_hi=200, rows_per_seq=3, k=16, n_layers=2, seed=1)
+    inp = make_decode(spec)
+    g = O.group_decode(inp)
+    for b in range(2):
+        n = int(inp["ctx"][b])
+        kv = O.paged_rows(inp["KV"][1], inp["KV_scale"][1], inp["block_table"][b], n)
+        for r in range(3):
+            o, _ = O.sparse_mla_row(O.bf16_to_f64(inp["Q"][1][b * 3 + r]), kv, g["idx"][b], inp["softmax_scale"])
+            assert np.array_equal(o, g["O"][1][b * 3 + r])
+        assert (g["idx"][b] < n).all()
+
+
+def test_paged_rows_follow_block_table():
+    spec = DecodeSpec("t", batch=3, ctx_lo=65, ctx_hi=300, rows_per_seq=1, k=8, n_layers=1, seed=2)
+    inp = make_decode(spec)
+    bt = inp["block_table"]
+    used = np.concatenate([bt[b, :(int(inp["ctx"][b]) + 63) // 64] for b in range(3)])
+    assert sorted(used) == list(range(inp["n_pages"]))          # a permutation of the pool
+    rows = O.paged_rows(inp["KV"][0], inp["KV_scale"][0], bt[1], 130)
+    p, s = bt[1][129 // 64], 129 % 64
+    assert np.array_equal(rows[129], O.e4m3_to_f64(inp["KV"][0][p, s]) * float(inp["KV_scale"][0][p, s]))
+
+
+def test_schedule_matches_pages():
+    sch = O.layer_schedule(GOLD["n_layers"]["value"])
+    full = [l for l, f, _ in sch if f]
+    assert full[:5] == GOLD["full_layers_0based_printed"]["value"]
+    assert full[-1] == GOLD["full_layers_0based_printed"]["last"]
+    assert len(full) == GOLD["n_full"]["value"]
+    shared = [l for l, f, _ in sch if not f]
+    assert len(shared) == GOLD["n_shared"]["value"]
+    assert round(100 * len(shared) / len(sch), 1) == GOLD["shared_fraction_pct"]["value"]
+    for l, f, p in sch:
+        assert sch[p][1] and 0 <= l - p <= 3 and (f == (p == l))
+
+
+def test_param_arithmetic_matches_pages():
+    assert O.indexer_param_count() == GOLD["params_per_indexer"]["value"]
+    assert GOLD["n_shared"]["value"] * O.indexer_param_count() == GOLD["params_removed"]["value"]
+
+
+# ----------------------------------------------------------------------------- planted mistakes
+
+
+def _mutant(fn, old, new):
+    src = inspect.getsource(fn)
+    assert old in src, (old, fn.__name__)
+    ns = dict(vars(O))
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)
+    return ns[fn.__name__]
+
+
+@pytest.mark.parametrize("old,new", [
+    ("np.maximum(x, 0.0)", "x"),                 # dropped ReLU
+    ("w[t] @ np.maximum", "w[0] @ np.maximum"),  # wrong query row of the weights
+    ("k[:n].T", "k[:n][::-1].T"),               # reversed key order
+])
+def test_planted_indexer_mistakes_are_caught(old, new):
+    bad = _mutant(O.indexer_scores, old, new)
+    with pytest.raises(AssertionError):
+        test_indexer_closed_form_unit_vectors(bad)
+
+
+@pytest.mark.parametrize("old,new", [
+    ("np.arange(n), -s", "-np.arange(n), -s"),   # ties to the higher index
+    ("order[:min(k, n)]", "order[1:min(k, n) + 1]"),
+])
+def test_planted_topk_mistakes_are_caught(old, new):
+    bad = _mutant(O.topk_row, old, new)
+    with pytest.raises(AssertionError):
+        test_topk_brute_force_tiny(bad)
+
+
+@pytest.mark.parametrize("old,new", [
+    ("softmax_scale * (Q @ kv.T)", "(Q @ kv.T)"),       # dropped scale
+    ("kv[:, :D_V]", "kv[:, -D_V:]"),                    # value from the wrong dims
+    ("sel = sel[sel >= 0]", "sel = np.abs(sel)"),        # padding not masked
+])
+def test_planted_attention_mistakes_are_caught(old, new):
+    bad = _mutant(O.sparse_mla_row, old, new)
+    with pytest.raises(AssertionError):
+        test_sparse_equals_dense_when_k_covers_history(bad)
