@@ -1,0 +1,702 @@
+// Host side of the C ABI declared in include/dsa.h: argument validation, tensor-map
+// encoding, launch configuration and the IndexShare group orchestration.  All device
+// memory is owned by the caller; the only library state is one device status word per
+// device, per-device launch attributes, and the thread-local error text.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/dsa.h"
+#include "indexer.cuh"
+#include "mla.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
+#include "topk.cuh"
+
+namespace dsa {
+
+__device__ int g_status_word;  // DEVERR_* bits, cleared by dsa_sync_status
+
+// Test hook: an mbarrier that expects two arrivals but gets one; the bounded wait runs out.
+__global__ void debug_wait_kernel(int* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 2);
+    fence_mbar_init();
+    mbar_arrive(smem_u32(&bar));
+    mbar_wait(smem_u32(&bar), 0, &abort_flag, status, limit_ns);
+  }
+}
+
+namespace {
+
+thread_local std::string t_err;
+int64_t g_wait_ns = 2000000000LL;
+std::atomic<int64_t> g_launches{0};
+
+void count_launch(int n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+void trace(void** ev, int i, cudaStream_t st) {
+  if (ev && ev[i]) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st);
+}
+
+dsa_status fail(dsa_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return s;
+}
+
+dsa_status cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return DSA_OK;
+  return fail(DSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define DSA_TRY(x)                       \
+  do {                                   \
+    const dsa_status _s = (x);           \
+    if (_s != DSA_OK) return _s;         \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceState {
+  bool ready = false;
+  int sms = 148;
+  int* status = nullptr;
+};
+DeviceState g_dev[64];
+std::mutex g_mu;
+
+dsa_status device_state(DeviceState** out) {
+  int dev = 0;
+  DSA_TRY(cuda_check(cudaGetDevice(&dev), "cudaGetDevice"));
+  if (dev < 0 || dev >= 64) return fail(DSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0;
+    DSA_TRY(cuda_check(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "attr"));
+    DSA_TRY(cuda_check(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev), "attr"));
+    if (major != 10 || minor != 0)
+      return fail(DSA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a only", dev,
+                  major, minor);
+    DSA_TRY(cuda_check(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev), "attr"));
+    void* sym = nullptr;
+    DSA_TRY(cuda_check(cudaGetSymbolAddress(&sym, g_status_word), "cudaGetSymbolAddress(status)"));
+    d.status = static_cast<int*>(sym);
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(idx::indexer_kernel<false, false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            idx::Cfg<false, false>::SMEM_BYTES),
+                       "smem attr"));
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(idx::indexer_kernel<true, false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            idx::Cfg<true, false>::SMEM_BYTES),
+                       "smem attr"));
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(idx::indexer_kernel<true, true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            idx::Cfg<true, true>::SMEM_BYTES),
+                       "smem attr"));
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES),
+                       "smem attr"));
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES),
+                       "smem attr"));
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(topk::topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(sizeof(topk::Smem))),
+                       "smem attr"));
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(topk::topk_seg_resolve_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(sizeof(topk::Smem))),
+                       "smem attr"));
+    d.ready = true;
+  }
+  *out = &d;
+  return DSA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D tiled map with 128-byte swizzle: [outer rows x inner elements], row stride in bytes.
+dsa_status make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer,
+                    uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                        const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return DSA_OK;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------- validation
+
+dsa_status check_view(const dsa_cache_view* v, int32_t dim, const char* name) {
+  if (!v) return fail(DSA_ERR_INVALID_ARG, "%s: null cache view", name);
+  if (!v->data || !aligned16(v->data)) return fail(DSA_ERR_INVALID_ARG, "%s: data null or not 16-byte aligned", name);
+  if (v->dim != dim) return fail(DSA_ERR_UNSUPPORTED, "%s: dim %d, expected %d", name, v->dim, dim);
+  if (v->dtype != DSA_BF16 && v->dtype != DSA_E4M3) return fail(DSA_ERR_INVALID_ARG, "%s: bad dtype", name);
+  const int64_t es = v->dtype == DSA_BF16 ? 2 : 1;
+  if (v->n_tokens < 0) return fail(DSA_ERR_INVALID_ARG, "%s: n_tokens < 0", name);
+  if (v->dtype == DSA_E4M3 && (!v->scale || !aligned16(v->scale)))
+    return fail(DSA_ERR_INVALID_ARG, "%s: e4m3 cache needs a 16-byte aligned scale array", name);
+  if (v->block_table) {
+    if (v->dtype != DSA_E4M3) return fail(DSA_ERR_UNSUPPORTED, "%s: paged caches must be e4m3", name);
+    if (v->row_stride != dim) return fail(DSA_ERR_INVALID_ARG, "%s: paged row_stride must equal dim", name);
+    if (!v->seq_lens) return fail(DSA_ERR_INVALID_ARG, "%s: paged cache needs seq_lens", name);
+    if (v->max_pages <= 0 || v->batch <= 0) return fail(DSA_ERR_INVALID_ARG, "%s: bad max_pages/batch", name);
+    if (v->n_tokens % DSA_PAGE) return fail(DSA_ERR_INVALID_ARG, "%s: n_tokens must be pages*64", name);
+    if (v->n_tokens / DSA_PAGE > INT32_MAX) return fail(DSA_ERR_INVALID_ARG, "%s: too many pages", name);
+  } else {
+    if (v->row_stride < dim || (v->row_stride * es) % 16)
+      return fail(DSA_ERR_INVALID_ARG, "%s: row_stride %lld invalid", name, static_cast<long long>(v->row_stride));
+    if (v->n_tokens > INT32_MAX) return fail(DSA_ERR_INVALID_ARG, "%s: n_tokens too large", name);
+  }
+  return DSA_OK;
+}
+
+// ---------------------------------------------------------------------------- launches
+
+dsa_status launch_indexer(const void* q, int32_t q_dtype, const float* q_scale, const float* w, int32_t n_q,
+                          int32_t q_pos0, const dsa_cache_view* keys, float* scores, int64_t ld,
+                          cudaStream_t st) {
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  const bool fp8 = q_dtype == DSA_E4M3;
+  const bool paged = keys->block_table != nullptr;
+  idx::Params p{};
+  p.q_scale = q_scale;
+  p.w = w;
+  p.key_scale = keys->scale;
+  p.block_table = keys->block_table;
+  p.seq_lens = keys->seq_lens;
+  p.scores = scores;
+  p.ld = ld;
+  p.n_tokens = keys->n_tokens;
+  p.n_q = n_q;
+  p.q_pos0 = q_pos0;
+  p.max_pages = keys->max_pages;
+  p.n_pages = static_cast<int32_t>(keys->n_tokens / DSA_PAGE);
+  p.status = ds->status;
+  p.wait_ns = static_cast<uint64_t>(g_wait_ns);
+  CUtensorMap mq, mk;
+  const uint64_t qrows = static_cast<uint64_t>(n_q) * 32;
+  if (paged) {
+    DSA_TRY(make_map(&mq, q, false, 128, qrows, 128, 128, 32));
+    DSA_TRY(make_map(&mk, keys->data, false, 128, static_cast<uint64_t>(keys->n_tokens), 128, 128, 64));
+    const int64_t max_len = static_cast<int64_t>(keys->max_pages) * DSA_PAGE;
+    const int64_t tiles = (max_len + idx::BLOCK_KEYS - 1) / idx::BLOCK_KEYS;
+    dim3 grid(static_cast<unsigned>((tiles + idx::UNIT_TILES - 1) / idx::UNIT_TILES), static_cast<unsigned>(n_q));
+    using C = idx::Cfg<true, true>;
+    idx::indexer_kernel<true, true><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, p);
+    count_launch();
+  } else {
+    const int64_t max_len = std::min<int64_t>(static_cast<int64_t>(q_pos0) + n_q, keys->n_tokens);
+    const int64_t tiles = (max_len + idx::BLOCK_KEYS - 1) / idx::BLOCK_KEYS;
+    if (tiles <= 0) return DSA_OK;
+    if (fp8) {
+      using C = idx::Cfg<true, false>;
+      DSA_TRY(make_map(&mq, q, false, 128, qrows, 128, 128, 256));
+      DSA_TRY(make_map(&mk, keys->data, false, 128, static_cast<uint64_t>(keys->n_tokens),
+                       static_cast<uint64_t>(keys->row_stride), 128, 128));
+      dim3 grid(static_cast<unsigned>((tiles + idx::UNIT_TILES - 1) / idx::UNIT_TILES),
+                static_cast<unsigned>((n_q + 15) / 16));
+      idx::indexer_kernel<true, false><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, p);
+      count_launch();
+    } else {
+      using C = idx::Cfg<false, false>;
+      DSA_TRY(make_map(&mq, q, true, 128, qrows, 256, 64, 256));
+      DSA_TRY(make_map(&mk, keys->data, true, 128, static_cast<uint64_t>(keys->n_tokens),
+                       static_cast<uint64_t>(keys->row_stride) * 2, 64, 128));
+      dim3 grid(static_cast<unsigned>((tiles + idx::UNIT_TILES - 1) / idx::UNIT_TILES),
+                static_cast<unsigned>((n_q + 15) / 16));
+      idx::indexer_kernel<false, false><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, p);
+      count_launch();
+    }
+  }
+  return cuda_check(cudaGetLastError(), "indexer launch");
+}
+
+// Top-k launch plan: row mode unless the rows are too few to fill the GPU and long.
+struct TopkPlan {
+  bool segmented = false;
+  int32_t segs = 1;
+  int32_t seg_len = 0;
+  int32_t gcap = 0;
+  size_t ws = 0;
+};
+
+TopkPlan plan_topk(int32_t n_rows, int64_t max_len, int32_t k, int sms) {
+  TopkPlan pl;
+  if (n_rows <= 0 || max_len <= k || n_rows >= 2 * sms || max_len <= 32768) return pl;
+  pl.segmented = true;
+  const int64_t by_len = (max_len + 8191) / 8192;  // at least 8K candidates per segment
+  int64_t segs = (4LL * sms + n_rows - 1) / n_rows;
+  segs = std::max<int64_t>(1, std::min(segs, by_len));
+  pl.segs = static_cast<int32_t>(segs);
+  pl.seg_len = static_cast<int32_t>(align_up(static_cast<size_t>((max_len + segs - 1) / segs), 4));
+  pl.gcap = static_cast<int32_t>(std::max<int64_t>(topk::CAND_CAP, std::min<int64_t>(max_len, 1 << 16)));
+  pl.ws = static_cast<size_t>(n_rows) * (topk::BINS * 4 + 16 + static_cast<size_t>(pl.gcap) * 8) + 256;
+  return pl;
+}
+
+dsa_status launch_topk(const float* scores, int64_t ld, int32_t n_rows, const int32_t* row_len,
+                       int64_t causal_len0, int64_t max_len, int32_t k, int32_t* idx_out, void* ws,
+                       size_t ws_bytes, cudaStream_t st) {
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  const int64_t cap = std::min(ld, max_len);
+  const TopkPlan pl = plan_topk(n_rows, cap, k, ds->sms);
+  if (!pl.segmented) {
+    topk::topk_row_kernel<<<n_rows, topk::THREADS, sizeof(topk::Smem), st>>>(scores, ld, n_rows, row_len,
+                                                                             causal_len0, cap, k, idx_out);
+    count_launch();
+    return cuda_check(cudaGetLastError(), "topk launch");
+  }
+  if (!ws || ws_bytes < pl.ws)
+    return fail(DSA_ERR_WORKSPACE, "topk needs %zu workspace bytes, got %zu", pl.ws, ws_bytes);
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  topk::SegWs sw;
+  sw.hist = reinterpret_cast<uint32_t*>(b);
+  sw.counters = reinterpret_cast<int32_t*>(b + static_cast<size_t>(n_rows) * topk::BINS * 4);
+  const size_t head = static_cast<size_t>(n_rows) * (topk::BINS * 4 + 16);
+  sw.cand_key = reinterpret_cast<uint32_t*>(b + head);
+  sw.cand_idx = reinterpret_cast<int32_t*>(b + head + static_cast<size_t>(n_rows) * pl.gcap * 4);
+  sw.gcap = pl.gcap;
+  DSA_TRY(cuda_check(cudaMemsetAsync(ws, 0, head, st), "topk workspace clear"));
+  dim3 grid(pl.segs, n_rows);
+  topk::topk_seg_hist_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k,
+                                                                 pl.seg_len, sw);
+  topk::topk_seg_filter_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k,
+                                                                   pl.seg_len, sw, idx_out);
+  topk::topk_seg_resolve_kernel<<<n_rows, topk::THREADS, sizeof(topk::Smem), st>>>(scores, ld, row_len,
+                                                                                  causal_len0, cap, k, sw, idx_out);
+  count_launch(3);
+  return cuda_check(cudaGetLastError(), "topk launch");
+}
+
+int32_t mla_splits(int32_t n_q, int32_t k, int sms) {
+  const int32_t tiles = (k + mla::TILE - 1) / mla::TILE;
+  if (n_q >= sms || tiles <= 1) return 1;
+  int32_t s = (sms + n_q - 1) / n_q;
+  s = std::min(s, tiles);
+  // balance: equal tiles per split
+  const int32_t tps = (tiles + s - 1) / s;
+  return (tiles + tps - 1) / tps;
+}
+
+size_t mla_ws_bytes(int32_t n_q, int32_t k, int sms) {
+  const int32_t s = mla_splits(n_q, k, sms);
+  if (s <= 1) return 0;
+  return static_cast<size_t>(n_q) * s * (64 * 512 * 4 + 128 * 4) + 256;
+}
+
+dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* idx, int32_t n_q, int32_t rpi,
+                      int32_t k, float softmax_scale, void* out, float* lse, void* ws, size_t ws_bytes,
+                      cudaStream_t st) {
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  if (n_q == 0) return DSA_OK;
+  const bool paged = kv->block_table != nullptr;
+  mla::Params p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.kv = static_cast<const uint8_t*>(kv->data);
+  p.kv_scale = kv->scale;
+  p.block_table = kv->block_table;
+  p.seq_lens = kv->seq_lens;
+  p.idx = idx;
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.row_stride = kv->row_stride;
+  p.n_tokens = kv->n_tokens;
+  p.n_q = n_q;
+  p.rows_per_idx = rpi;
+  p.k = k;
+  p.max_pages = kv->max_pages;
+  p.n_pages = static_cast<int32_t>(kv->n_tokens / DSA_PAGE);
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.status = ds->status;
+  p.wait_ns = static_cast<uint64_t>(g_wait_ns);
+  p.n_split = mla_splits(n_q, k, ds->sms);
+  if (p.n_split > 1) {
+    const size_t need = mla_ws_bytes(n_q, k, ds->sms);
+    if (!ws || ws_bytes < need) return fail(DSA_ERR_WORKSPACE, "sparse MLA needs %zu workspace bytes", need);
+    p.part_o = static_cast<float*>(ws);
+    p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                         static_cast<size_t>(n_q) * p.n_split * 64 * 512 * 4);
+  }
+  const unsigned grid = static_cast<unsigned>(n_q) * p.n_split;
+  if (paged)
+    mla::sparse_mla_kernel<true><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
+  else
+    mla::sparse_mla_kernel<false><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
+  count_launch();
+  DSA_TRY(cuda_check(cudaGetLastError(), "sparse MLA launch"));
+  if (p.n_split > 1) {
+    mla::combine_kernel<<<dim3(n_q, 64), 128, 0, st>>>(p.part_o, p.part_ml, p.n_split, p.out, p.lse);
+    count_launch();
+    DSA_TRY(cuda_check(cudaGetLastError(), "combine launch"));
+  }
+  return DSA_OK;
+}
+
+// ---------------------------------------------------------------------------- group plan
+
+struct GroupPlan {
+  bool quant_q = false, quant_k = false;
+  size_t off_q8 = 0, off_sq = 0, off_k8 = 0, off_sk = 0, off_scores = 0, off_topk = 0, off_mla = 0, total = 0;
+  int32_t chunk_rows = 0;
+  int64_t ld = 0;
+  int64_t max_len = 0;
+  size_t topk_ws = 0;
+};
+
+constexpr int64_t kScoreBudgetFloats = 16LL << 20;  // 64 MB of scores per chunk (L2-sized)
+
+dsa_status plan_group(const dsa_group_args* a, int sms, GroupPlan* g) {
+  const dsa_cache_view& kv = a->idx_keys;
+  const bool paged = kv.block_table != nullptr;
+  const int64_t n = a->n_idx_rows;
+  g->quant_q = a->indexer_dtype == DSA_E4M3;
+  g->quant_k = a->indexer_dtype == DSA_E4M3 && kv.dtype == DSA_BF16;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  if (g->quant_q) {
+    g->off_q8 = take(static_cast<size_t>(n) * 32 * 128);
+    g->off_sq = take(static_cast<size_t>(n) * 32 * 4);
+  }
+  if (g->quant_k) {
+    g->off_k8 = take(static_cast<size_t>(kv.n_tokens) * 128);
+    g->off_sk = take(static_cast<size_t>(kv.n_tokens) * 4);
+  }
+  if (paged) {
+    g->max_len = static_cast<int64_t>(kv.max_pages) * DSA_PAGE;
+    g->ld = g->max_len;
+    g->chunk_rows = static_cast<int32_t>(n);
+  } else {
+    g->max_len = std::min<int64_t>(static_cast<int64_t>(a->q_pos0) + n, kv.n_tokens);
+    g->ld = static_cast<int64_t>(align_up(static_cast<size_t>(std::max<int64_t>(g->max_len, 4)), 4));
+    int64_t c = std::max<int64_t>(16, kScoreBudgetFloats / g->ld);
+    c = c / 16 * 16;
+    g->chunk_rows = static_cast<int32_t>(std::min<int64_t>(c, n));
+  }
+  g->off_scores = take(static_cast<size_t>(g->chunk_rows) * g->ld * 4);
+  g->topk_ws = plan_topk(g->chunk_rows, g->max_len, a->k, sms).ws;
+  g->off_topk = take(g->topk_ws);
+  size_t mla_ws = 0;
+  const int32_t nq = a->n_idx_rows * a->q_rows_per_idx_row;
+  mla_ws = mla_ws_bytes(nq, a->k, sms);
+  g->off_mla = take(mla_ws);
+  g->total = off;
+  return DSA_OK;
+}
+
+dsa_status check_group(const dsa_group_args* a) {
+  if (!a) return fail(DSA_ERR_INVALID_ARG, "null group args");
+  if (a->n_layers < 1 || a->n_layers > DSA_GROUP_MAX_LAYERS)
+    return fail(DSA_ERR_INVALID_ARG, "n_layers %d not in [1,4]", a->n_layers);
+  if (a->k < 1 || a->k > DSA_MAX_K) return fail(DSA_ERR_INVALID_ARG, "k %d not in [1,2048]", a->k);
+  if (a->n_idx_rows < 0 || a->q_rows_per_idx_row < 1) return fail(DSA_ERR_INVALID_ARG, "bad row counts");
+  if (a->indexer_dtype != DSA_BF16 && a->indexer_dtype != DSA_E4M3)
+    return fail(DSA_ERR_INVALID_ARG, "bad indexer_dtype");
+  DSA_TRY(check_view(&a->idx_keys, 128, "idx_keys"));
+  if (a->indexer_dtype == DSA_BF16 && a->idx_keys.dtype != DSA_BF16)
+    return fail(DSA_ERR_UNSUPPORTED, "bf16 indexer needs bf16 keys");
+  if (a->idx_keys.block_table && a->idx_keys.batch != a->n_idx_rows)
+    return fail(DSA_ERR_INVALID_ARG, "paged indexer keys: batch %d != n_idx_rows %d", a->idx_keys.batch,
+                a->n_idx_rows);
+  if (!a->q_idx || !aligned16(a->q_idx) || !a->w || !aligned16(a->w))
+    return fail(DSA_ERR_INVALID_ARG, "q_idx / w null or misaligned");
+  for (int l = 0; l < a->n_layers; ++l) {
+    DSA_TRY(check_view(&a->kv[l], 576, "kv"));
+    if (!a->q[l] || !aligned16(a->q[l]) || !a->out[l] || !aligned16(a->out[l]))
+      return fail(DSA_ERR_INVALID_ARG, "layer %d: q/out null or misaligned", l);
+    if (a->lse[l] && !aligned16(a->lse[l])) return fail(DSA_ERR_INVALID_ARG, "layer %d: lse misaligned", l);
+    if (!a->kv[l].block_table && a->kv[l].dtype != DSA_BF16)
+      return fail(DSA_ERR_UNSUPPORTED, "dense latent caches must be bf16");
+    if (a->kv[l].block_table && a->kv[l].batch != a->n_idx_rows)
+      return fail(DSA_ERR_INVALID_ARG, "layer %d: paged batch != n_idx_rows", l);
+  }
+  return DSA_OK;
+}
+
+}  // namespace
+}  // namespace dsa
+
+using namespace dsa;
+
+// ================================================================================= C ABI
+
+extern "C" {
+
+int32_t dsa_abi_version(void) { return DSA_ABI_VERSION; }
+
+size_t dsa_abi_sizeof(int32_t which) {
+  switch (which) {
+    case 0: return sizeof(dsa_cache_view);
+    case 1: return sizeof(dsa_index_handle);
+    case 2: return sizeof(dsa_group_args);
+  }
+  return 0;
+}
+
+const char* dsa_status_str(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported";
+    case DSA_ERR_STALE_HANDLE: return "stale index handle";
+    case DSA_ERR_TIMEOUT: return "device wait timed out";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_WORKSPACE: return "workspace too small";
+    case DSA_ERR_BOUNDS: return "index or page out of range";
+  }
+  return "unknown status";
+}
+
+const char* dsa_last_error(void) { return t_err.c_str(); }
+
+int64_t dsa_launch_count(void) { return g_launches.load(); }
+
+int64_t dsa_set_wait_limit_ns(int64_t ns) {
+  const int64_t old = g_wait_ns;
+  if (ns > 0) g_wait_ns = ns;
+  return old;
+}
+
+int32_t dsa_layer_is_full(int32_t layer) { return layer >= 0 && (layer < 2 || (layer - 2) % 4 == 0) ? 1 : 0; }
+int32_t dsa_layer_producer(int32_t layer) {
+  if (layer < 0) return -1;
+  if (dsa_layer_is_full(layer)) return layer;
+  return 2 + 4 * ((layer - 2) / 4);
+}
+
+dsa_status dsa_sync_status(void* stream) {
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  DSA_TRY(cuda_check(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "cudaStreamSynchronize"));
+  int v = 0;
+  DSA_TRY(cuda_check(cudaMemcpy(&v, ds->status, sizeof(int), cudaMemcpyDeviceToHost), "read status"));
+  const int zero = 0;
+  DSA_TRY(cuda_check(cudaMemcpy(ds->status, &zero, sizeof(int), cudaMemcpyHostToDevice), "clear status"));
+  if (v & DEVERR_TIMEOUT) return fail(DSA_ERR_TIMEOUT, "a bounded device wait ran out");
+  if (v & DEVERR_BOUNDS) return fail(DSA_ERR_BOUNDS, "a kernel skipped an out-of-range index or page");
+  return DSA_OK;
+}
+
+dsa_status dsa_debug_bounded_wait(int64_t timeout_ns, void* stream) {
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  if (timeout_ns <= 0 || timeout_ns > 10000000000LL) return fail(DSA_ERR_INVALID_ARG, "timeout out of range");
+  debug_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ds->status,
+                                                                      static_cast<uint64_t>(timeout_ns));
+  count_launch();
+  return cuda_check(cudaGetLastError(), "debug wait launch");
+}
+
+dsa_status dsa_quant_e4m3(const void* x_bf16, int64_t n_vec, int32_t vec_len, uint8_t* codes, float* scale,
+                          void* stream) {
+  if (vec_len != 128) return fail(DSA_ERR_UNSUPPORTED, "vec_len %d (only 128)", vec_len);
+  if (n_vec < 0) return fail(DSA_ERR_INVALID_ARG, "n_vec < 0");
+  if (n_vec == 0) return DSA_OK;
+  if (!x_bf16 || !codes || !scale || !aligned16(x_bf16) || !aligned16(codes) || !aligned16(scale))
+    return fail(DSA_ERR_INVALID_ARG, "null or misaligned pointer");
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  const int64_t blocks = (n_vec + 7) / 8;
+  if (blocks > INT32_MAX) return fail(DSA_ERR_INVALID_ARG, "n_vec too large");
+  quant_e4m3_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(x_bf16), n_vec, codes, scale);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "quant launch");
+}
+
+dsa_status dsa_indexer_score(const void* q, int32_t q_dtype, const float* q_scale, const float* w, int32_t n_q,
+                             int32_t q_pos0, const dsa_cache_view* keys, float* scores, int64_t ld_scores,
+                             void* stream) {
+  DSA_TRY(check_view(keys, 128, "keys"));
+  if (n_q < 0 || q_pos0 < 0) return fail(DSA_ERR_INVALID_ARG, "n_q / q_pos0 negative");
+  if (n_q == 0) return DSA_OK;
+  if (q_dtype != keys->dtype) return fail(DSA_ERR_UNSUPPORTED, "q dtype must equal key dtype");
+  if (!q || !aligned16(q) || !w || !aligned16(w) || !scores || !aligned16(scores))
+    return fail(DSA_ERR_INVALID_ARG, "q / w / scores null or misaligned");
+  if (q_dtype == DSA_E4M3 && (!q_scale || !aligned16(q_scale)))
+    return fail(DSA_ERR_INVALID_ARG, "e4m3 queries need q_scale");
+  if (ld_scores <= 0 || ld_scores % 4) return fail(DSA_ERR_INVALID_ARG, "ld_scores must be a positive multiple of 4");
+  if (keys->block_table) {
+    if (keys->batch != n_q) return fail(DSA_ERR_INVALID_ARG, "paged keys: batch != n_q");
+    if (ld_scores < static_cast<int64_t>(keys->max_pages) * DSA_PAGE)
+      return fail(DSA_ERR_INVALID_ARG, "ld_scores < max_pages*64");
+  } else {
+    if (ld_scores < std::min<int64_t>(static_cast<int64_t>(q_pos0) + n_q, keys->n_tokens))
+      return fail(DSA_ERR_INVALID_ARG, "ld_scores shorter than the longest row");
+  }
+  return launch_indexer(q, q_dtype, q_scale, w, n_q, q_pos0, keys, scores, ld_scores,
+                        static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_topk_workspace_bytes(int32_t n_rows, int64_t max_len, int32_t k) {
+  DeviceState* ds = nullptr;
+  if (device_state(&ds) != DSA_OK) return 0;
+  return plan_topk(n_rows, max_len, k, ds->sms).ws;
+}
+
+dsa_status dsa_topk(const float* scores, int64_t ld, int32_t n_rows, const int32_t* row_len, int64_t causal_len0,
+                    int64_t max_len, int32_t k, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  if (k < 1 || k > DSA_MAX_K) return fail(DSA_ERR_INVALID_ARG, "k %d not in [1,2048]", k);
+  if (n_rows < 0 || ld <= 0 || ld % 4 || max_len < 0 || ld > INT32_MAX)
+    return fail(DSA_ERR_INVALID_ARG, "bad n_rows / ld / max_len");
+  if (n_rows == 0) return DSA_OK;
+  if (!scores || !aligned16(scores) || !idx_out || !aligned16(idx_out))
+    return fail(DSA_ERR_INVALID_ARG, "scores / idx_out null or misaligned");
+  if (!row_len && causal_len0 < 0) return fail(DSA_ERR_INVALID_ARG, "causal_len0 < 0");
+  return launch_topk(scores, ld, n_rows, row_len, causal_len0, max_len, k, idx_out, workspace, workspace_bytes,
+                     static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_sparse_mla_workspace_bytes(int32_t n_q, int32_t k, const dsa_cache_view* kv) {
+  (void)kv;
+  DeviceState* ds = nullptr;
+  if (device_state(&ds) != DSA_OK) return 0;
+  return mla_ws_bytes(n_q, k, ds->sms);
+}
+
+dsa_status dsa_sparse_mla_attn(const void* q, const dsa_cache_view* kv, const int32_t* idx, int32_t n_q,
+                               int32_t q_rows_per_idx_row, int32_t k, float softmax_scale, void* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  DSA_TRY(check_view(kv, 576, "kv"));
+  if (k < 1 || k > DSA_MAX_K) return fail(DSA_ERR_INVALID_ARG, "k %d not in [1,2048]", k);
+  if (n_q < 0 || q_rows_per_idx_row < 1 || n_q % q_rows_per_idx_row)
+    return fail(DSA_ERR_INVALID_ARG, "n_q must be a non-negative multiple of q_rows_per_idx_row");
+  if (n_q == 0) return DSA_OK;
+  if (!q || !aligned16(q) || !idx || !aligned16(idx) || !out || !aligned16(out))
+    return fail(DSA_ERR_INVALID_ARG, "q / idx / out null or misaligned");
+  if (lse && !aligned16(lse)) return fail(DSA_ERR_INVALID_ARG, "lse misaligned");
+  if (!(softmax_scale > 0.f)) return fail(DSA_ERR_INVALID_ARG, "softmax_scale must be > 0");
+  if (kv->block_table) {
+    if (kv->batch != n_q / q_rows_per_idx_row)
+      return fail(DSA_ERR_INVALID_ARG, "paged kv: batch != n_q / q_rows_per_idx_row");
+  } else if (kv->dtype != DSA_BF16) {
+    return fail(DSA_ERR_UNSUPPORTED, "dense latent caches must be bf16");
+  }
+  return launch_mla(q, kv, idx, n_q, q_rows_per_idx_row, k, softmax_scale, out, lse, workspace, workspace_bytes,
+                    static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_group_workspace_bytes(const dsa_group_args* a) {
+  if (check_group(a) != DSA_OK) return 0;
+  DeviceState* ds = nullptr;
+  if (device_state(&ds) != DSA_OK) return 0;
+  GroupPlan g;
+  plan_group(a, ds->sms, &g);
+  return g.total;
+}
+
+dsa_status indexshare_group_forward(const dsa_group_args* a, dsa_index_handle* h, int32_t reuse_only,
+                                    void* stream) {
+  DSA_TRY(check_group(a));
+  if (!h || !h->idx || !aligned16(h->idx)) return fail(DSA_ERR_INVALID_ARG, "null handle or handle buffer");
+  if (h->rows != a->n_idx_rows || h->k != a->k) {
+    if (reuse_only)
+      return fail(DSA_ERR_STALE_HANDLE, "handle holds %d x %d indices, call needs %d x %d", h->rows, h->k,
+                  a->n_idx_rows, a->k);
+    return fail(DSA_ERR_INVALID_ARG, "handle buffer is %d x %d, call needs %d x %d", h->rows, h->k, a->n_idx_rows,
+                a->k);
+  }
+  if (reuse_only && !h->filled) return fail(DSA_ERR_STALE_HANDLE, "reuse of an unfilled index handle");
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  GroupPlan g;
+  DSA_TRY(plan_group(a, ds->sms, &g));
+  if (g.total > 0 && (!a->workspace || a->workspace_bytes < g.total))
+    return fail(DSA_ERR_WORKSPACE, "group needs %zu workspace bytes, got %zu", g.total, a->workspace_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+  const int32_t n = a->n_idx_rows;
+  void** ev = a->trace_events;
+  trace(ev, 0, st);
+  if (!reuse_only && n > 0) {
+    // a1: FP8 prep
+    const void* qi = a->q_idx;
+    const float* qs = nullptr;
+    dsa_cache_view keys = a->idx_keys;
+    if (g.quant_q) {
+      DSA_TRY(dsa_quant_e4m3(a->q_idx, static_cast<int64_t>(n) * 32, 128, ws + g.off_q8,
+                             reinterpret_cast<float*>(ws + g.off_sq), st));
+      qi = ws + g.off_q8;
+      qs = reinterpret_cast<const float*>(ws + g.off_sq);
+    }
+    if (g.quant_k) {
+      if (keys.row_stride != 128) return fail(DSA_ERR_UNSUPPORTED, "bf16 keys to quantise must be contiguous");
+      DSA_TRY(dsa_quant_e4m3(keys.data, keys.n_tokens, 128, ws + g.off_k8,
+                             reinterpret_cast<float*>(ws + g.off_sk), st));
+      keys.data = ws + g.off_k8;
+      keys.scale = reinterpret_cast<const float*>(ws + g.off_sk);
+      keys.dtype = DSA_E4M3;
+      keys.row_stride = 128;
+    }
+    const int32_t qdt = g.quant_q ? DSA_E4M3 : DSA_BF16;
+    float* scores = reinterpret_cast<float*>(ws + g.off_scores);
+    const bool paged = keys.block_table != nullptr;
+    const size_t qrow_bytes = qdt == DSA_E4M3 ? 32 * 128 : 32 * 128 * 2;
+    for (int32_t c0 = 0; c0 < n; c0 += g.chunk_rows) {
+      const int32_t cn = std::min(g.chunk_rows, n - c0);
+      const uint8_t* qc = static_cast<const uint8_t*>(qi) + static_cast<size_t>(c0) * qrow_bytes;
+      const float* qsc = qs ? qs + static_cast<size_t>(c0) * 32 : nullptr;
+      DSA_TRY(launch_indexer(qc, qdt, qsc, a->w + static_cast<size_t>(c0) * 32, cn, a->q_pos0 + c0, &keys, scores,
+                             g.ld, st));
+      DSA_TRY(launch_topk(scores, g.ld, cn, paged ? keys.seq_lens : nullptr,
+                          static_cast<int64_t>(a->q_pos0) + c0 + 1, g.max_len, a->k,
+                          h->idx + static_cast<size_t>(c0) * a->k, ws + g.off_topk, g.topk_ws, st));
+    }
+    h->generation += 1;
+    h->filled = 1;
+    h->producer_layer = a->first_layer;
+  }
+  trace(ev, 1, st);
+  const int32_t nq = n * a->q_rows_per_idx_row;
+  for (int l = 0; l < a->n_layers; ++l) {
+    trace(ev, 2 + 2 * l, st);
+    DSA_TRY(launch_mla(a->q[l], &a->kv[l], h->idx, nq, a->q_rows_per_idx_row, a->k, a->softmax_scale, a->out[l],
+                       a->lse[l], ws + g.off_mla, g.total - g.off_mla, st));
+    trace(ev, 3 + 2 * l, st);
+  }
+  return DSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,356 @@
+// Step a4: exact per-row Top-k by radix selection on CUDA cores.
+//
+// Each candidate s of a row gets the 64-bit composite key  (f32_key(score) << 32) | ~s,
+// so "larger composite" means "larger score, then lower position"; composites are unique
+// and the Top-k set is the k largest composites.  Selection walks six digits of the
+// composite (12, 12, 8 bits of the score key, then 12, 12, 8 bits of ~s).  At each digit
+// a histogram over the elements still matching the chosen prefix gives the bin T that
+// contains the k_rem-th largest; elements above T are emitted, the prefix is extended by
+// T, and the walk stops as soon as the elements matching the prefix are exactly k_rem.
+//
+// Row mode (one CTA per row): the row is read twice from global memory (histogram of the
+// first digit, then emit / collect the threshold bin into shared memory); later digits
+// run on the shared-memory candidates.  Segmented mode (few long rows): several CTAs per
+// row build the first-digit histogram and emit / collect in parallel through a global
+// workspace; one CTA per row then resolves the remaining digits.
+#pragma once
+#include "ptx.cuh"
+
+namespace dsa {
+namespace topk {
+
+constexpr int THREADS = 1024;
+constexpr int BINS = 4096;
+constexpr int CAND_CAP = 6144;  // shared-memory candidates of the threshold bin
+constexpr int SEG_THREADS = 512;
+
+struct Smem {
+  uint32_t hist[BINS];
+  uint32_t cand_key[CAND_CAP];
+  int32_t cand_idx[CAND_CAP];
+  uint32_t warp_sum[32];
+  int32_t out_cnt;
+  int32_t cand_cnt;
+  uint32_t sel_bin;
+  uint32_t sel_above;
+  uint32_t sel_eq;
+};
+
+__device__ __forceinline__ uint64_t composite(uint32_t key, int32_t idx) {
+  return (static_cast<uint64_t>(key) << 32) | static_cast<uint64_t>(~static_cast<uint32_t>(idx));
+}
+__device__ __forceinline__ int digit_shift(int lvl) {
+  // levels: bits [52,64), [40,52), [32,40), [20,32), [8,20), [0,8)
+  const int sh[6] = {52, 40, 32, 20, 8, 0};
+  return sh[lvl];
+}
+__device__ __forceinline__ int digit_bits(int lvl) { return (lvl == 2 || lvl == 5) ? 8 : 12; }
+
+// Block-wide: find bin T with above(T) < k_rem <= above(T) + hist[T], above(T) = sum of
+// bins > T.  Writes sel_bin / sel_above / sel_eq.  All threads of the block must call.
+template <int NT>
+__device__ void find_threshold(const uint32_t* hist, uint32_t k_rem, uint32_t* warp_sum, uint32_t* sel_bin,
+                               uint32_t* sel_above, uint32_t* sel_eq) {
+  constexpr int PER = BINS / NT;
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  uint32_t v = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) v += hist[t * PER + i];
+  uint32_t incl = v;  // sum over lanes >= lane
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
+    if (lane + off < 32) incl += y;
+  }
+  if (lane == 0) warp_sum[w] = incl;
+  __syncthreads();
+  uint32_t above_warp = 0;
+  for (int u = w + 1; u < NT / 32; ++u) above_warp += warp_sum[u];
+  const uint32_t excl = incl - v + above_warp;  // sum of bins owned by higher threads
+  if (excl < k_rem && k_rem <= excl + v) {
+    uint32_t acc = excl;
+    for (int i = PER - 1; i >= 0; --i) {
+      const uint32_t h = hist[t * PER + i];
+      if (acc + h >= k_rem) {
+        *sel_bin = t * PER + i;
+        *sel_above = acc;
+        *sel_eq = h;
+        break;
+      }
+      acc += h;
+    }
+  }
+  __syncthreads();
+}
+
+// Element sources for the digit walk.
+struct RowSrc {
+  const float* p;
+  int32_t n;
+  __device__ __forceinline__ int32_t size() const { return n; }
+  __device__ __forceinline__ uint64_t comp(int32_t i) const { return composite(f32_key(p[i]), i); }
+  __device__ __forceinline__ int32_t index(int32_t i) const { return i; }
+};
+struct CandSrc {
+  const uint32_t* keys;
+  const int32_t* idx;
+  int32_t n;
+  __device__ __forceinline__ int32_t size() const { return n; }
+  __device__ __forceinline__ uint64_t comp(int32_t i) const { return composite(keys[i], idx[i]); }
+  __device__ __forceinline__ int32_t index(int32_t i) const { return idx[i]; }
+};
+
+// Walk digits lvl0..5 over `src`, emitting into out[0..k) through the shared counter.
+template <int NT, class Src>
+__device__ void walk_digits(const Src& src, int lvl0, uint64_t pfx, uint64_t pmask, uint32_t k_rem, Smem& sm,
+                            int32_t* out, int32_t kmax) {
+  const int t = threadIdx.x;
+  for (int lvl = lvl0; lvl < 6 && k_rem > 0; ++lvl) {
+    const int sh = digit_shift(lvl);
+    const uint32_t dmask = (1u << digit_bits(lvl)) - 1u;
+    for (int b = t; b < BINS; b += NT) sm.hist[b] = 0;
+    __syncthreads();
+    const int32_t n = src.size();
+    for (int32_t i = t; i < n; i += NT) {
+      const uint64_t c = src.comp(i);
+      if ((c & pmask) == pfx) atomicAdd(&sm.hist[(c >> sh) & dmask], 1u);
+    }
+    __syncthreads();
+    find_threshold<NT>(sm.hist, k_rem, sm.warp_sum, &sm.sel_bin, &sm.sel_above, &sm.sel_eq);
+    const uint32_t T = sm.sel_bin, above = sm.sel_above, eq = sm.sel_eq;
+    const uint64_t new_pfx = pfx | (static_cast<uint64_t>(T) << sh);
+    const uint64_t new_mask = pmask | (static_cast<uint64_t>(dmask) << sh);
+    const bool take_eq = (eq == k_rem - above);
+    for (int32_t i = t; i < n; i += NT) {
+      const uint64_t c = src.comp(i);
+      if ((c & pmask) != pfx) continue;
+      const uint32_t d = static_cast<uint32_t>((c >> sh) & dmask);
+      if (d > T || (take_eq && d == T)) {
+        const int32_t pos = atomicAdd(&sm.out_cnt, 1);
+        if (pos < kmax) out[pos] = src.index(i);
+      }
+    }
+    __syncthreads();
+    if (take_eq) break;
+    k_rem -= above;
+    pfx = new_pfx;
+    pmask = new_mask;
+  }
+}
+
+// Candidates of row r: row_len[r] (device array) or causal_len0 + r, capped at `cap`.
+__device__ __forceinline__ int32_t row_length(int32_t r, const int32_t* row_len, int64_t causal_len0, int64_t cap) {
+  int64_t n = row_len ? static_cast<int64_t>(row_len[r]) : causal_len0 + r;
+  n = n < 0 ? 0 : n;
+  return static_cast<int32_t>(n > cap ? cap : n);
+}
+
+// ------------------------------------------------------------------------------- row mode
+
+__global__ void __launch_bounds__(THREADS) topk_row_kernel(const float* __restrict__ scores, int64_t ld,
+                                                           int32_t n_rows, const int32_t* __restrict__ row_len,
+                                                           int64_t causal_len0, int64_t cap, int32_t k,
+                                                           int32_t* __restrict__ idx_out) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  const int32_t r = blockIdx.x;
+  if (r >= n_rows) return;
+  const int t = threadIdx.x;
+  const float* row = scores + static_cast<int64_t>(r) * ld;
+  int32_t* out = idx_out + static_cast<int64_t>(r) * k;
+  const int32_t n = row_length(r, row_len, causal_len0, cap);
+  if (t == 0) {
+    sm.out_cnt = 0;
+    sm.cand_cnt = 0;
+  }
+  if (n <= k) {
+    for (int32_t i = t; i < k; i += THREADS) out[i] = i < n ? i : -1;
+    return;
+  }
+  for (int b = t; b < BINS; b += THREADS) sm.hist[b] = 0;
+  __syncthreads();
+  // pass 1: histogram of the top 12 key bits (vectorised, row start is 16-byte aligned)
+  const int32_t n4 = n & ~3;
+  for (int32_t i = t * 4; i < n4; i += THREADS * 4) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(row + i));
+    atomicAdd(&sm.hist[f32_key(v.x) >> 20], 1u);
+    atomicAdd(&sm.hist[f32_key(v.y) >> 20], 1u);
+    atomicAdd(&sm.hist[f32_key(v.z) >> 20], 1u);
+    atomicAdd(&sm.hist[f32_key(v.w) >> 20], 1u);
+  }
+  for (int32_t i = n4 + t; i < n; i += THREADS) atomicAdd(&sm.hist[f32_key(row[i]) >> 20], 1u);
+  __syncthreads();
+  find_threshold<THREADS>(sm.hist, static_cast<uint32_t>(k), sm.warp_sum, &sm.sel_bin, &sm.sel_above, &sm.sel_eq);
+  const uint32_t T = sm.sel_bin, above = sm.sel_above, eq = sm.sel_eq;
+  const uint32_t k_rem = static_cast<uint32_t>(k) - above;
+  const bool take_eq = (eq == k_rem);
+  const bool collect = !take_eq && eq <= static_cast<uint32_t>(CAND_CAP);
+  // pass 2: emit bins above T, collect bin T
+  auto visit = [&](float f, int32_t i) {
+    const uint32_t key = f32_key(f);
+    const uint32_t d = key >> 20;
+    if (d > T || (take_eq && d == T)) {
+      const int32_t pos = atomicAdd(&sm.out_cnt, 1);
+      if (pos < k) out[pos] = i;
+    } else if (collect && d == T) {
+      const int32_t c = atomicAdd(&sm.cand_cnt, 1);
+      if (c < CAND_CAP) {
+        sm.cand_key[c] = key;
+        sm.cand_idx[c] = i;
+      }
+    }
+  };
+  for (int32_t i = t * 4; i < n4; i += THREADS * 4) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(row + i));
+    visit(v.x, i);
+    visit(v.y, i + 1);
+    visit(v.z, i + 2);
+    visit(v.w, i + 3);
+  }
+  for (int32_t i = n4 + t; i < n; i += THREADS) visit(row[i], i);
+  __syncthreads();
+  if (take_eq) return;
+  const uint64_t pfx = static_cast<uint64_t>(T) << 52;
+  const uint64_t pmask = static_cast<uint64_t>(0xFFF) << 52;
+  if (collect) {
+    CandSrc src{sm.cand_key, sm.cand_idx, min(sm.cand_cnt, CAND_CAP)};
+    walk_digits<THREADS>(src, 1, pfx, pmask, k_rem, sm, out, k);
+  } else {
+    RowSrc src{row, n};
+    walk_digits<THREADS>(src, 1, pfx, pmask, k_rem, sm, out, k);
+  }
+}
+
+// --------------------------------------------------------------------------- segmented mode
+// Workspace per row: hist[4096] u32, counters[4] i32 (out, cand), then cand keys/idx [gcap].
+
+struct SegWs {
+  uint32_t* hist;     // [rows][BINS]
+  int32_t* counters;  // [rows][4]
+  uint32_t* cand_key; // [rows][gcap]
+  int32_t* cand_idx;  // [rows][gcap]
+  int32_t gcap;
+};
+
+__global__ void __launch_bounds__(SEG_THREADS) topk_seg_hist_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                    const int32_t* __restrict__ row_len,
+                                                                    int64_t causal_len0, int64_t cap, int32_t k,
+                                                                    int32_t seg_len, SegWs ws) {
+  __shared__ uint32_t hist[BINS];
+  const int32_t r = blockIdx.y;
+  const int32_t n = row_length(r, row_len, causal_len0, cap);
+  if (n <= k) return;
+  const int32_t beg = blockIdx.x * seg_len;
+  if (beg >= n) return;
+  const int32_t end = min(n, beg + seg_len);
+  const int t = threadIdx.x;
+  for (int b = t; b < BINS; b += SEG_THREADS) hist[b] = 0;
+  __syncthreads();
+  const float* row = scores + static_cast<int64_t>(r) * ld;
+  for (int32_t i = beg + t * 4; i + 3 < end; i += SEG_THREADS * 4) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(row + i));
+    atomicAdd(&hist[f32_key(v.x) >> 20], 1u);
+    atomicAdd(&hist[f32_key(v.y) >> 20], 1u);
+    atomicAdd(&hist[f32_key(v.z) >> 20], 1u);
+    atomicAdd(&hist[f32_key(v.w) >> 20], 1u);
+  }
+  const int32_t tail = beg + ((end - beg) & ~3);
+  for (int32_t i = tail + t; i < end; i += SEG_THREADS) atomicAdd(&hist[f32_key(row[i]) >> 20], 1u);
+  __syncthreads();
+  uint32_t* g = ws.hist + static_cast<int64_t>(r) * BINS;
+  for (int b = t; b < BINS; b += SEG_THREADS)
+    if (hist[b]) atomicAdd(&g[b], hist[b]);
+}
+
+__global__ void __launch_bounds__(SEG_THREADS) topk_seg_filter_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                      const int32_t* __restrict__ row_len,
+                                                                      int64_t causal_len0, int64_t cap, int32_t k,
+                                                                      int32_t seg_len, SegWs ws,
+                                                                      int32_t* __restrict__ idx_out) {
+  __shared__ uint32_t hist[BINS];
+  __shared__ uint32_t warp_sum[32];
+  __shared__ uint32_t sel[3];
+  const int32_t r = blockIdx.y;
+  const int32_t n = row_length(r, row_len, causal_len0, cap);
+  if (n <= k) return;
+  const int32_t beg = blockIdx.x * seg_len;
+  if (beg >= n) return;
+  const int32_t end = min(n, beg + seg_len);
+  const int t = threadIdx.x;
+  const uint32_t* g = ws.hist + static_cast<int64_t>(r) * BINS;
+  for (int b = t; b < BINS; b += SEG_THREADS) hist[b] = g[b];
+  __syncthreads();
+  find_threshold<SEG_THREADS>(hist, static_cast<uint32_t>(k), warp_sum, &sel[0], &sel[1], &sel[2]);
+  const uint32_t T = sel[0], above = sel[1], eq = sel[2];
+  const bool take_eq = (eq == static_cast<uint32_t>(k) - above);
+  const bool collect = !take_eq && eq <= static_cast<uint32_t>(ws.gcap);
+  const float* row = scores + static_cast<int64_t>(r) * ld;
+  int32_t* out = idx_out + static_cast<int64_t>(r) * k;
+  int32_t* cnt = ws.counters + static_cast<int64_t>(r) * 4;
+  uint32_t* ck = ws.cand_key + static_cast<int64_t>(r) * ws.gcap;
+  int32_t* ci = ws.cand_idx + static_cast<int64_t>(r) * ws.gcap;
+  for (int32_t i = beg + t; i < end; i += SEG_THREADS) {
+    const uint32_t key = f32_key(row[i]);
+    const uint32_t d = key >> 20;
+    if (d > T || (take_eq && d == T)) {
+      const int32_t pos = atomicAdd(&cnt[0], 1);
+      if (pos < k) out[pos] = i;
+    } else if (collect && d == T) {
+      const int32_t c = atomicAdd(&cnt[1], 1);
+      if (c < ws.gcap) {
+        ck[c] = key;
+        ci[c] = i;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(THREADS) topk_seg_resolve_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                   const int32_t* __restrict__ row_len,
+                                                                   int64_t causal_len0, int64_t cap, int32_t k,
+                                                                   SegWs ws, int32_t* __restrict__ idx_out) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  const int32_t r = blockIdx.x;
+  const int t = threadIdx.x;
+  const int32_t n = row_length(r, row_len, causal_len0, cap);
+  int32_t* out = idx_out + static_cast<int64_t>(r) * k;
+  if (n <= k) {
+    for (int32_t i = t; i < k; i += THREADS) out[i] = i < n ? i : -1;
+    return;
+  }
+  const uint32_t* g = ws.hist + static_cast<int64_t>(r) * BINS;
+  for (int b = t; b < BINS; b += THREADS) sm.hist[b] = g[b];
+  __syncthreads();
+  find_threshold<THREADS>(sm.hist, static_cast<uint32_t>(k), sm.warp_sum, &sm.sel_bin, &sm.sel_above, &sm.sel_eq);
+  const uint32_t T = sm.sel_bin, above = sm.sel_above, eq = sm.sel_eq;
+  const uint32_t k_rem = static_cast<uint32_t>(k) - above;
+  if (eq == k_rem) return;  // the filter pass emitted everything
+  if (t == 0) sm.out_cnt = static_cast<int32_t>(above);
+  const int32_t* cnt = ws.counters + static_cast<int64_t>(r) * 4;
+  const uint64_t pfx = static_cast<uint64_t>(T) << 52;
+  const uint64_t pmask = static_cast<uint64_t>(0xFFF) << 52;
+  const uint32_t* ck = ws.cand_key + static_cast<int64_t>(r) * ws.gcap;
+  const int32_t* ci = ws.cand_idx + static_cast<int64_t>(r) * ws.gcap;
+  if (eq <= static_cast<uint32_t>(CAND_CAP)) {
+    const int32_t c = min(cnt[1], CAND_CAP);
+    for (int32_t i = t; i < c; i += THREADS) {
+      sm.cand_key[i] = ck[i];
+      sm.cand_idx[i] = ci[i];
+    }
+    __syncthreads();
+    CandSrc src{sm.cand_key, sm.cand_idx, c};
+    walk_digits<THREADS>(src, 1, pfx, pmask, k_rem, sm, out, k);
+  } else if (eq <= static_cast<uint32_t>(ws.gcap)) {
+    __syncthreads();
+    CandSrc src{ck, ci, min(cnt[1], ws.gcap)};
+    walk_digits<THREADS>(src, 1, pfx, pmask, k_rem, sm, out, k);
+  } else {
+    __syncthreads();
+    RowSrc src{scores + static_cast<int64_t>(r) * ld, n};
+    walk_digits<THREADS>(src, 1, pfx, pmask, k_rem, sm, out, k);
+  }
+}
+
+}  // namespace topk
+}  // namespace dsa

@@ -221,18 +221,22 @@ def group_prefill(inp: dict, rows, fp8_indexer: bool = False, idx_override=None)
     L, k = inp["L"], inp["k"]
     rows = list(rows)
     if fp8_indexer:
-        q8, sq = quantize_e4m3_rows(inp["q_idx"], IDX_DIM)
         k8, sk = quantize_e4m3_rows(inp["k_idx"], IDX_DIM)
-        qv = e4m3_to_f64(q8) * sq.reshape(L, IDX_HEADS, 1)
-        kv = e4m3_to_f64(k8) * sk.reshape(L, 1)
+        kv = e4m3_to_f64(k8) * sk.reshape(-1, 1)
     else:
-        qv = bf16_to_f64(inp["q_idx"])
         kv = bf16_to_f64(inp["k_idx"])
-    w = np.asarray(inp["w"], dtype=np.float64)
+
+    def query(t):  # indexer query of row t (only the rows asked for are converted)
+        if fp8_indexer:
+            q8, sq = quantize_e4m3_rows(np.asarray(inp["q_idx"][t])[None], IDX_DIM)
+            return e4m3_to_f64(q8) * sq.reshape(1, IDX_HEADS, 1)
+        return bf16_to_f64(np.asarray(inp["q_idx"][t])[None])
+
     idx = {}
     if idx_override is None:
         for t in rows:
-            sc = indexer_scores(qv[t:t + 1], w[t:t + 1], kv, [t + 1])[0]
+            wt = np.asarray(inp["w"][t], dtype=np.float64)[None]
+            sc = indexer_scores(query(t), wt, kv, [t + 1])[0]
             idx[t] = topk_row(sc, t + 1, k)
     else:
         idx = {t: np.asarray(idx_override[t]) for t in rows}

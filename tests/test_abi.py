@@ -1,0 +1,121 @@
+"""The C-ABI library loads, exports every declared symbol and validates arguments (CPU only).
+
+No compute call is made here: the checks below all fail host-side validation before any
+CUDA call, or are pure host functions.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_sparse_11_b200 as dsa
+from long_context_sparse_11_b200 import binding as B
+import oracle.dsa_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b([a-z_][a-z0-9_]*)\s*\([^;{]*\)\s*;", src)
+    return sorted(set(n for n in names if n.startswith(("dsa_", "indexshare_"))))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_sparse_11_b200.build import build
+    build()
+    return dsa.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(B.EXPORTS)
+
+
+def test_struct_layouts_match(lib):
+    assert lib.dsa_abi_version() == 1
+    assert lib.dsa_abi_sizeof(0) == ctypes.sizeof(B.CacheView)
+    assert lib.dsa_abi_sizeof(1) == ctypes.sizeof(B.IndexHandle)
+    assert lib.dsa_abi_sizeof(2) == ctypes.sizeof(B.GroupArgs)
+
+
+def test_schedule_agrees_with_oracle(lib):
+    for l, full, prod in O.layer_schedule(78):
+        assert bool(lib.dsa_layer_is_full(l)) == full
+        assert lib.dsa_layer_producer(l) == prod
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert lib.dsa_status_str(s)
+
+
+def _err(lib):
+    return lib.dsa_last_error().decode()
+
+
+def test_host_validation_rejects_before_launch(lib):
+    # vec_len other than 128
+    assert lib.dsa_quant_e4m3(16, 4, 64, 16, 16, None) == B.DSA_ERR_UNSUPPORTED
+    # misaligned pointers
+    assert lib.dsa_quant_e4m3(17, 4, 128, 16, 16, None) == B.DSA_ERR_INVALID_ARG
+    assert "aligned" in _err(lib)
+    # k out of range
+    assert lib.dsa_topk(16, 64, 4, None, 1, 64, 0, 16, None, 0, None) == B.DSA_ERR_INVALID_ARG
+    assert lib.dsa_topk(16, 64, 4, None, 1, 64, 4096, 16, None, 0, None) == B.DSA_ERR_INVALID_ARG
+    # ld not a multiple of 4
+    assert lib.dsa_topk(16, 63, 4, None, 1, 63, 8, 16, None, 0, None) == B.DSA_ERR_INVALID_ARG
+    # wrong cache dims / dtypes
+    v = B.CacheView(16, None, None, None, 128, 100, 64, B.DSA_BF16, 0, 0)
+    assert lib.dsa_indexer_score(16, 0, None, 16, 4, 0, ctypes.byref(v), 16, 128, None) == B.DSA_ERR_UNSUPPORTED
+    v = B.CacheView(16, None, None, None, 128, 100, 128, B.DSA_BF16, 0, 0)
+    assert lib.dsa_indexer_score(16, B.DSA_E4M3, None, 16, 4, 0, ctypes.byref(v), 16, 128, None) \
+        == B.DSA_ERR_UNSUPPORTED
+    # paged caches must be e4m3 and carry seq_lens
+    v = B.CacheView(16, None, 32, None, 576, 6400, 576, B.DSA_BF16, 4, 2)
+    assert lib.dsa_sparse_mla_attn(16, ctypes.byref(v), 16, 2, 1, 8, 0.04, 16, None, None, 0, None) \
+        == B.DSA_ERR_UNSUPPORTED
+    v = B.CacheView(16, 48, 32, None, 576, 6400, 576, B.DSA_E4M3, 4, 2)
+    assert lib.dsa_sparse_mla_attn(16, ctypes.byref(v), 16, 2, 1, 8, 0.04, 16, None, None, 0, None) \
+        == B.DSA_ERR_INVALID_ARG
+    # n_q not a multiple of the rows per index row
+    v = B.CacheView(16, None, None, None, 576, 100, 576, B.DSA_BF16, 0, 0)
+    assert lib.dsa_sparse_mla_attn(16, ctypes.byref(v), 16, 5, 2, 8, 0.04, 16, None, None, 0, None) \
+        == B.DSA_ERR_INVALID_ARG
+
+
+def test_group_handle_checks(lib):
+    a = B.GroupArgs()
+    a.q_idx, a.w = 16, 32
+    a.idx_keys = B.CacheView(16, None, None, None, 128, 100, 128, B.DSA_BF16, 0, 0)
+    a.indexer_dtype, a.n_idx_rows, a.k, a.q_rows_per_idx_row, a.n_layers = B.DSA_BF16, 100, 64, 1, 2
+    a.softmax_scale = 0.04
+    for i in range(2):
+        a.q[i], a.out[i] = 64, 128
+        a.kv[i] = B.CacheView(16, None, None, None, 576, 100, 576, B.DSA_BF16, 0, 0)
+    # handle of the wrong size for a reuse call: stale
+    h = B.IndexHandle(256, 100, 32, 1, 0, 1)
+    assert lib.indexshare_group_forward(ctypes.byref(a), ctypes.byref(h), 1, None) == B.DSA_ERR_STALE_HANDLE
+    # unfilled handle for a reuse call: stale
+    h = B.IndexHandle(256, 100, 64, 0, -1, 0)
+    assert lib.indexshare_group_forward(ctypes.byref(a), ctypes.byref(h), 1, None) == B.DSA_ERR_STALE_HANDLE
+    assert "unfilled" in _err(lib)
+    # too many layers
+    a.n_layers = 5
+    assert lib.indexshare_group_forward(ctypes.byref(a), ctypes.byref(h), 0, None) == B.DSA_ERR_INVALID_ARG
+
+
+def test_product_path_never_imports_oracle():
+    pkg = os.path.join(ROOT, "long_context_sparse_11_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in txt.lower(), f

@@ -1,0 +1,143 @@
+"""IndexShare group (Full layer + Shared layers) through the C ABI against the fp64 oracle.
+
+Covers the 512-token tiny prefill workload in full, a scaled FP8-indexer prefill, a
+scaled batched decode with MTP rows and paged FP8 caches, and the reuse-handle rules.
+Tolerances as in test_gpu_kernels.py; the FP8 indexer path also checks end-to-end
+relative L2 <= 3e-2 against the oracle run on unquantised bf16 inputs.
+"""
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import long_context_sparse_11_b200 as dsa  # noqa: E402
+import oracle.dsa_oracle as O  # noqa: E402
+from synth import make_prefill, make_decode, PrefillSpec, DecodeSpec, WORKLOADS  # noqa: E402
+from test_gpu_kernels import (bf16_dev, u8_dev, f32_dev, i32_dev, bf16_host, check_topk_sets,  # noqa: E402
+                              attn_errors)
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from long_context_sparse_11_b200.build import build
+    build()
+    return dsa.load()
+
+
+def run_prefill_group(inp, fp8=False):
+    L, k = inp["L"], inp["k"]
+    kv = [bf16_dev(x) for x in inp["KV"]]
+    g = dsa.IndexShareGroup(bf16_dev(inp["q_idx"]), f32_dev(inp["w"]), dsa.dense_view(bf16_dev(inp["k_idx"])), k,
+                            [bf16_dev(x) for x in inp["Q"]], [dsa.dense_view(x) for x in kv],
+                            inp["softmax_scale"], indexer_dtype=dsa.DSA_E4M3 if fp8 else dsa.DSA_BF16)
+    out, lse = g.forward()
+    dsa.sync_status()
+    return g, [O.bf16_to_f64(bf16_host(o)) for o in out], [x.cpu().numpy() for x in lse]
+
+
+def oracle_scores_row(inp, t, fp8):
+    if fp8:
+        q8, sq = O.quantize_e4m3_rows(inp["q_idx"][t:t + 1], 128)
+        k8, sk = O.quantize_e4m3_rows(inp["k_idx"], 128)
+        qv = O.e4m3_to_f64(q8) * sq.reshape(1, 32, 1)
+        kv = O.e4m3_to_f64(k8) * sk.reshape(-1, 1)
+    else:
+        qv, kv = O.bf16_to_f64(inp["q_idx"][t:t + 1]), O.bf16_to_f64(inp["k_idx"])
+    return O.indexer_scores(qv, inp["w"][t:t + 1], kv, [t + 1])[0]
+
+
+def test_tiny_prefill_group_full():
+    inp = make_prefill(WORKLOADS["tiny_prefill"])
+    g, outs, lses = run_prefill_group(inp)
+    idx = g.idx.cpu().numpy()
+    L, k = inp["L"], inp["k"]
+    swaps = 0
+    for t in range(L):
+        swaps += check_topk_sets(idx[t], oracle_scores_row(inp, t, False), t + 1, k)
+    assert g.handle.filled == 1 and g.handle.generation == 1
+    rows = list(range(0, L, 5)) + [L - 1]
+    for l in range(4):                     # every layer attends over the Full layer's indices
+        KV = O.bf16_to_f64(inp["KV"][l])
+        for t in rows:
+            ref, rl = O.sparse_mla_row(O.bf16_to_f64(inp["Q"][l][t]), KV, idx[t], inp["softmax_scale"])
+            ma, rel = attn_errors(outs[l][t], ref)
+            assert ma <= 2e-2 and rel <= 5e-3, (l, t, ma, rel)
+            assert np.max(np.abs(lses[l][t] - rl)) <= 2e-3
+    print(f"tiny prefill: {swaps} tolerated Top-k swaps over {L} rows")
+
+
+def test_shared_layers_reuse_handle_without_indexer():
+    inp = make_prefill(PrefillSpec("t", L=700, k=64, seed=77))
+    g, outs, _ = run_prefill_group(inp)
+    idx0 = g.idx.clone()
+    # a reuse-only call must not touch the indices and must reproduce the outputs
+    g.idx.view(torch.int32)  # same buffer
+    out2, _ = g.forward(reuse_only=True)
+    dsa.sync_status()
+    assert torch.equal(g.idx, idx0)
+    assert g.handle.generation == 1
+    for l in range(4):
+        assert np.array_equal(O.bf16_to_f64(bf16_host(out2[l])), outs[l])
+
+
+def test_fp8_indexer_prefill_group():
+    spec = PrefillSpec("fp8", L=1500, k=256, seed=3, indexer_fp8=True)
+    inp = make_prefill(spec)
+    g, outs, _ = run_prefill_group(inp, fp8=True)
+    idx = g.idx.cpu().numpy()
+    L, k = inp["L"], inp["k"]
+    for t in range(0, L, 3):               # exact-set check against the oracle on dequantised inputs
+        check_topk_sets(idx[t], oracle_scores_row(inp, t, True), t + 1, k)
+    # end-to-end: the oracle runs the whole FP8-indexer group on the same inputs (its own
+    # quantisation and selection); relative L2 over the sampled outputs <= 3e-2
+    rows = list(range(k, L, 37))
+    ref = O.group_prefill(inp, rows, fp8_indexer=True)
+    num = den = 0.0
+    for l in range(4):
+        for t in rows:
+            num += np.sum((outs[l][t] - ref["O"][l][t]) ** 2)
+            den += np.sum(ref["O"][l][t] ** 2)
+    rel = math.sqrt(num / den)
+    assert rel <= 3e-2, rel
+    # informational: what FP8 quantisation itself changes against the bf16 indexer
+    ref16 = O.group_prefill(inp, rows, fp8_indexer=False)
+    overlap = np.mean([len(set(ref16["idx"][t]) & set(ref["idx"][t])) / k for t in rows])
+    print(f"fp8 group: end-to-end rel L2 {rel:.2e}; oracle fp8-vs-bf16 Top-k overlap {overlap:.3f}")
+
+
+def test_decode_group_mtp_paged():
+    spec = DecodeSpec("d", batch=6, ctx_lo=500, ctx_hi=20000, rows_per_seq=5, k=512, n_layers=4, seed=8)
+    inp = make_decode(spec)
+    ctx, bt = inp["ctx"], inp["block_table"]
+    ctx_d, bt_d = i32_dev(ctx), i32_dev(bt)
+    keys = dsa.paged_view(u8_dev(inp["idx_keys"]), f32_dev(inp["idx_key_scale"]), bt_d, ctx_d)
+    kvs = [dsa.paged_view(u8_dev(inp["KV"][l]), f32_dev(inp["KV_scale"][l]), bt_d, ctx_d) for l in range(4)]
+    g = dsa.IndexShareGroup(bf16_dev(inp["q_idx"]), f32_dev(inp["w"]), keys, spec.k,
+                            [bf16_dev(x) for x in inp["Q"]], kvs, inp["softmax_scale"],
+                            indexer_dtype=dsa.DSA_E4M3, q_rows_per_idx_row=spec.rows_per_seq)
+    out, lse = g.forward()
+    dsa.sync_status()
+    idx = g.idx.cpu().numpy()
+    q8, sq = O.quantize_e4m3_rows(inp["q_idx"], 128)
+    qv = O.e4m3_to_f64(q8) * sq.reshape(-1, 32, 1)
+    for b in range(spec.batch):
+        n = int(ctx[b])
+        kk = O.paged_rows(inp["idx_keys"], inp["idx_key_scale"], bt[b], n)
+        sc = O.indexer_scores(qv[b:b + 1], inp["w"][b:b + 1], kk, [n])[0]
+        check_topk_sets(idx[b], sc, n, spec.k)
+    outs = [O.bf16_to_f64(bf16_host(o)) for o in out]
+    for l in range(4):
+        for b in range(spec.batch):
+            kv = O.paged_rows(inp["KV"][l], inp["KV_scale"][l], bt[b], int(ctx[b]))
+            for r in range(spec.rows_per_seq):
+                row = b * spec.rows_per_seq + r
+                ref, _ = O.sparse_mla_row(O.bf16_to_f64(inp["Q"][l][row]), kv, idx[b], inp["softmax_scale"])
+                ma, rel = attn_errors(outs[l][row], ref)
+                assert ma <= 2e-2 and rel <= 5e-3, (l, row, ma, rel)
