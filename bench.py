@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of one DSA + IndexShare step on B200: query tokens/s per IndexShare group.
+
+A step is one IndexShare group on one batch of synthetic input: the Full layer's indexer
+scores + Top-k into the reuse handle, then sparse MLA for the Full layer and its 3 Shared
+layers.  Default workload: causal prefill of 32,768 tokens, Top-2048, bf16, AR(1)-drifting
+indexer keys.  Inputs are generated on the device by the seeded generator before timing.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One JSON line is printed by rank 0.  Multi-GPU (torchrun): every rank runs its own
+independent group (weak scaling, no collective on the data path); the time is the max over
+ranks of the CUDA-event time.  ``--impl reference`` times the fp64 CPU oracle on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "query tokens/s per IndexShare group"
+UNIT = "query tokens/s"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--workload", default="prefill_32k",
+                   choices=["tiny_prefill", "prefill_32k", "prefill_128k_fp8", "decode_b32_mtp4"])
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
+    p.add_argument("--ref-seconds", type=float, default=150.0, help="reference arm total budget")
+    p.add_argument("--seq-len", type=int, default=None, help="override L of a prefill workload (profiling)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- distributed
+
+
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        if args.impl == "ours":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=600))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- workload
+
+
+def workload_config(name, seq_len=None):
+    import dataclasses
+    from synth import WORKLOADS
+    spec = WORKLOADS[name]
+    if seq_len is not None and hasattr(spec, "L"):
+        spec = dataclasses.replace(spec, L=seq_len)
+    if name.startswith("decode"):
+        return spec, {"workload": name, "batch": spec.batch, "context": f"U[{spec.ctx_lo},{spec.ctx_hi}]",
+                      "rows_per_seq": spec.rows_per_seq, "k": spec.k, "layers_per_group": 4,
+                      "cache": "paged e4m3, 64-token pages", "indexer": "e4m3"}
+    return spec, {"workload": name, "seq_len": spec.L, "k": spec.k, "layers_per_group": spec.n_layers,
+                  "indexer": "e4m3" if spec.indexer_fp8 else "bf16", "latent_kv": "bf16 [L,576]",
+                  "heads": 64, "indexer_heads": 32}
+
+
+def algorithmic_counts(spec, ctx=None):
+    """Algorithmic work of one group: indexer flops, MLA flops per layer, tokens per step."""
+    if hasattr(spec, "L"):
+        L, k = spec.L, spec.k
+        pairs = L * (L + 1) // 2
+        sel = sum(min(k, t + 1) for t in range(L))
+        return {"tokens": L, "indexer_flops": 8192.0 * pairs, "mla_flops_per_layer": 139264.0 * sel,
+                "mla_rows": L}
+    import numpy as np
+    ctx = np.asarray(ctx)
+    R = spec.rows_per_seq
+    sel = float(np.minimum(ctx, spec.k).sum())
+    return {"tokens": len(ctx) * R, "indexer_flops": 8192.0 * float(ctx.sum()),
+            "mla_flops_per_layer": 139264.0 * sel * R, "mla_rows": len(ctx) * R,
+            "indexer_bytes": 132.0 * float(ctx.sum())}
+
+
+def build_group(spec, name, dev):
+    """Device inputs and an IndexShareGroup for the workload."""
+    import torch
+    import long_context_sparse_11_b200 as dsa
+    from synth import make_prefill, make_decode
+    if name.startswith("decode"):
+        inp = make_decode(spec, device=dev)
+        ctx_d = torch.from_numpy(inp["ctx"].astype("int32")).to(dev)
+        bt_d = torch.from_numpy(inp["block_table"]).to(dev)
+        keys = dsa.paged_view(inp["idx_keys"], inp["idx_key_scale"], bt_d, ctx_d)
+        kvs = [dsa.paged_view(inp["KV"][l], inp["KV_scale"][l], bt_d, ctx_d) for l in range(4)]
+        g = dsa.IndexShareGroup(inp["q_idx"], inp["w"], keys, spec.k, inp["Q"], kvs, inp["softmax_scale"],
+                                indexer_dtype=dsa.DSA_E4M3, q_rows_per_idx_row=spec.rows_per_seq)
+        return g, inp
+    inp = make_prefill(spec, device=dev)
+    g = dsa.IndexShareGroup(inp["q_idx"], inp["w"], dsa.dense_view(inp["k_idx"]), spec.k, inp["Q"],
+                            [dsa.dense_view(x) for x in inp["KV"]], inp["softmax_scale"],
+                            indexer_dtype=dsa.DSA_E4M3 if spec.indexer_fp8 else dsa.DSA_BF16)
+    return g, inp
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_smi_id(dev_index):
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev_index).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[dev_index]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+
+
+def oracle_rows_per_second(spec, name, inp, budget_s, seed_rows=0):
+    """Time the fp64 oracle on a bounded sample of rows of the same workload (host cores)."""
+    import numpy as np
+    import oracle.dsa_oracle as O
+    import torch
+
+    def host_bits(t):
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+    if name.startswith("decode"):
+        host = {"ctx": inp["ctx"], "block_table": inp["block_table"], "k": spec.k, "rows_per_seq": spec.rows_per_seq,
+                "softmax_scale": spec.softmax_scale, "q_idx": host_bits(inp["q_idx"]), "w": inp["w"].cpu().numpy(),
+                "idx_keys": inp["idx_keys"].cpu().numpy(), "idx_key_scale": inp["idx_key_scale"].cpu().numpy(),
+                "Q": [host_bits(q) for q in inp["Q"]], "KV": [x.cpu().numpy() for x in inp["KV"]],
+                "KV_scale": [x.cpu().numpy() for x in inp["KV_scale"]]}
+        order = list(np.random.default_rng(seed_rows).permutation(len(inp["ctx"])))
+        done, t0 = 0, time.perf_counter()
+        while order and time.perf_counter() - t0 < budget_s:
+            O.group_decode(host, seqs=[order.pop()])
+            done += spec.rows_per_seq
+        el = time.perf_counter() - t0
+        return done / el, f"{done // spec.rows_per_seq} whole sequences (all {spec.rows_per_seq} rows, 4 layers)", el
+    L = spec.L
+    host = {"L": L, "k": spec.k, "softmax_scale": spec.softmax_scale, "k_idx": host_bits(inp["k_idx"]),
+            "q_idx": _LazyRows(inp["q_idx"]), "w": _LazyRows(inp["w"], bf16=False),
+            "Q": [_LazyRows(q) for q in inp["Q"]], "KV": [host_bits(x) for x in inp["KV"]]}
+    rng = np.random.default_rng(seed_rows)
+    # one oracle call over a batch of uniformly drawn rows, sized from a short calibration
+    n, el = 2, 0.0
+    for _ in range(6):
+        rows = sorted(int(r) for r in rng.integers(0, L, size=n))
+        t0 = time.perf_counter()
+        O.group_prefill(host, rows, fp8_indexer=spec.indexer_fp8)
+        el = time.perf_counter() - t0
+        if el >= 0.5 * budget_s:
+            break
+        n = max(n + 1, int(n * min(8.0, budget_s / max(el, 1e-3))))
+    return n / el, f"{n} uniformly drawn query rows in one oracle call (indexer + Top-k + 4 layers each)", el
+
+
+class _LazyRows:
+    """Row access to a device tensor for the oracle (copies one row to the host on demand)."""
+
+    def __init__(self, t, bf16=True):
+        self.t, self.bf16 = t, bf16
+
+    def __getitem__(self, i):
+        import numpy as np
+        import torch
+        r = self.t[i]
+        if self.bf16:
+            return r.view(torch.int16).cpu().numpy().view(np.uint16)
+        return r.cpu().numpy()
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        th = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        th = 1
+    return max(1, min(th, len(os.sched_getaffinity(0))))
+
+
+# ----------------------------------------------------------------------------- arms
+
+
+def run_ours(args, ws, rank, local):
+    import torch
+    import long_context_sparse_11_b200 as dsa
+    from long_context_sparse_11_b200.build import build
+
+    build()
+    lib = dsa.load()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    spec, cfg = workload_config(args.workload, args.seq_len)
+    g, inp = build_group(spec, args.workload, dev)
+    counts = algorithmic_counts(spec, inp.get("ctx"))
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.int32, device=dev)   # 1 GiB > 126 MB L2
+
+    # trace events: indexer phase and each layer's sparse MLA launch (recorded once so
+    # that torch creates the underlying CUDA events before their handles are passed on)
+    n_ev = 2 + 2 * 4
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    for e in evs:
+        e.record(stream)
+    torch.cuda.synchronize()
+    import ctypes
+    ev_arr = (ctypes.c_void_p * n_ev)(*[e.cuda_event for e in evs])
+    assert all(e.cuda_event for e in evs)
+
+    def step(traced):
+        g.args.trace_events = ctypes.cast(ev_arr, ctypes.c_void_p) if traced else None
+        g.forward()
+
+    for _ in range(args.warmup):
+        step(False)
+    dsa.sync_status()
+    barrier(ws)
+    torch.cuda.synchronize()
+    t_steps, mla_ms, idx_ms = [], [], []
+    n0 = lib.dsa_launch_count()
+    with ClockSampler(gpu_smi_id(local)) as clk:
+        for _ in range(args.steps):
+            flush.fill_(1)                                  # evict L2 between steps (untimed)
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            step(True)
+            s1.record(stream)
+            s1.synchronize()
+            t_steps.append(s0.elapsed_time(s1))
+            idx_ms.append(evs[0].elapsed_time(evs[1]))
+            mla_ms.extend(evs[2 + 2 * l].elapsed_time(evs[3 + 2 * l]) for l in range(4))
+    torch.cuda.synchronize()
+    launches = lib.dsa_launch_count() - n0
+    barrier(ws)
+    dsa.sync_status()
+    total_ms = max_over_ranks(sum(t_steps), ws)
+    ms_per_step = total_ms / args.steps
+    value = counts["tokens"] * ws / (total_ms / 1e3) * args.steps
+    clocks = clk.summary()
+
+    hbm, bf16_peak, peak_kind = measured_peaks()
+    mla_avg = statistics.mean(mla_ms)
+    achieved = counts["mla_flops_per_layer"] / (mla_avg / 1e3) / 1e12
+    roofline = {"kernel": "sparse_mla_kernel (a6)", "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(achieved / bf16_peak, 4),
+                "peak_source": f"{peak_kind} bf16 dense (burst)", "traffic": None,
+                "algorithmic_flops_per_launch": counts["mla_flops_per_layer"], "avg_launch_ms": round(mla_avg, 4)}
+    idx_avg = statistics.mean(idx_ms)
+    phases = {"indexer_topk_ms": round(idx_avg, 4), "mla_ms_per_layer": round(mla_avg, 4),
+              "indexer_topk_tflops": round(counts["indexer_flops"] / (idx_avg / 1e3) / 1e12, 1)}
+
+    # end to end through the public API: pinned host inputs -> device, group, outputs -> host
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, g, inp, spec, counts, stream, ws)
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline and ws == 1:
+        v, sample, el = oracle_rows_per_second(spec, args.workload, inp, args.cpu_seconds)
+        cpu = {"value": round(v, 3), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": sample,
+               "seconds": round(el, 1)}
+    if rank == 0:
+        cfg.update({"l2": "flushed (1 GiB write) between timed steps", "parallelism": f"replicas x{ws}"})
+        line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if not spec.__dict__.get("indexer_fp8")
+                else "bf16+e4m3", "data": "synthetic (seeded SplitMix64 normals)", "config": cfg,
+                "roofline": roofline, "phases": phases, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+                "clocks": clocks}
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, g, inp, spec, counts, stream, ws):
+    import torch
+    import long_context_sparse_11_b200 as dsa
+    dev_in = []
+    for key in ("q_idx", "w", "k_idx", "idx_keys", "idx_key_scale", "Q", "KV", "KV_scale"):
+        v = inp.get(key)
+        for x in (v if isinstance(v, list) else [v]):
+            if hasattr(x, "is_cuda") and x.is_cuda:
+                dev_in.append(x)
+    host_in = [t.cpu().pin_memory() for t in dev_in]
+    host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in g.out + g.lse]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    steps = max(2, min(args.steps, 5))
+
+    def one():
+        for h, d in zip(host_in, dev_in):
+            d.copy_(h, non_blocking=True)
+        g.forward()
+        for h, d in zip(host_out, g.out + g.lse):
+            h.copy_(d, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    e1.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), ws)
+    dsa.sync_status()
+    return {"value": round(counts["tokens"] * ws * steps / (ms / 1e3), 1), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 3)}
+
+
+def run_reference(args, ws, rank):
+    """fp64 oracle on the host cores: each step a bounded sample of the same workload."""
+    if rank != 0:
+        return
+    import torch
+    spec, cfg = workload_config(args.workload, args.seq_len)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    from synth import make_prefill, make_decode
+    if args.workload.startswith("decode"):
+        inp = make_decode(spec, device=dev)
+    else:
+        inp = make_prefill(spec, device=dev)
+    per_step = max(1.0, args.ref_seconds / (args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_rows_per_second(spec, args.workload, inp, per_step, seed_rows=99)
+    tot_rows, tot_s, sample = 0.0, 0.0, ""
+    for i in range(args.steps):
+        v, sample, el = oracle_rows_per_second(spec, args.workload, inp, per_step, seed_rows=i)
+        tot_rows += v * el
+        tot_s += el
+    value = tot_rows / tot_s
+    cfg.update({"parallelism": "host cores, rank 0 only"})
+    cpu = {"value": round(value, 3), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+           "sample": f"per step: {sample}, about {per_step:.1f} s"}
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded SplitMix64 normals)", "config": cfg, "cpu_baseline": cpu,
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    ws, rank, local = dist_setup(args)
+    if args.gpus != ws and ws > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {ws}", file=sys.stderr)
+    try:
+        if args.impl == "reference":
+            run_reference(args, ws, rank)
+        else:
+            run_ours(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

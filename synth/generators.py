@@ -133,6 +133,20 @@ def normal_torch(seed: int, start: int, n: int, device="cpu", chunk: int = 1 << 
     return out
 
 
+def normal_bf16_torch(seed: int, n: int, device, scale: float = 1.0, chunk: int = 1 << 25):
+    """bf16 tensor equal to bf16_bits_torch(normal_torch(seed, 0, n) * scale), built chunk
+    by chunk so that no float64 copy of the whole tensor is held."""
+    import torch
+    out = torch.empty(n, dtype=torch.bfloat16, device=device)
+    for a in range(0, n, chunk):
+        b = min(n, a + chunk)
+        x = normal_torch(seed, a, b - a, device=device, chunk=chunk)
+        if scale != 1.0:
+            x = x * scale
+        out[a:b] = bf16_bits_torch(x)
+    return out
+
+
 def bf16_bits_torch(x):
     """float64 tensor -> bf16 tensor with the same rounding as :func:`bf16_bits_np`."""
     import torch

@@ -23,7 +23,7 @@ import numpy as np
 
 from .generators import (
     normal_np, normal_torch, bf16_bits_np, bf16_bits_torch, sub_seed, ar1_keys_np,
-    uniform_np, e4m3_codes_torch, splitmix64_np,
+    uniform_np, e4m3_codes_torch, splitmix64_np, normal_bf16_torch,
 )
 
 __all__ = ["PrefillSpec", "DecodeSpec", "WORKLOADS", "make_prefill", "make_decode",
@@ -122,10 +122,15 @@ def make_prefill(spec: PrefillSpec, L: int | None = None, device=None, layers=No
     layers = range(spec.n_layers) if layers is None else layers
     out["Q"], out["KV"] = [], []
     for l in layers:
-        out["Q"].append(_bf16(_normal(sub_seed(s, l, T_Q), L * MLA_HEADS * D_QK, device), device)
-                        .reshape(L, MLA_HEADS, D_QK))
-        out["KV"].append(_bf16(_normal(sub_seed(s, l, T_KV), L * D_QK, device), device).reshape(L, D_QK))
+        out["Q"].append(_bf16_normal(sub_seed(s, l, T_Q), L * MLA_HEADS * D_QK, device).reshape(L, MLA_HEADS, D_QK))
+        out["KV"].append(_bf16_normal(sub_seed(s, l, T_KV), L * D_QK, device).reshape(L, D_QK))
     return out
+
+
+def _bf16_normal(seed, n, device):
+    if device is None:
+        return bf16_bits_np(normal_np(seed, 0, n))
+    return normal_bf16_torch(seed, n, device)
 
 
 def decode_context_lengths(spec: DecodeSpec) -> np.ndarray:
