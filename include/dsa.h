@@ -209,6 +209,31 @@ dsa_status indexshare_group_forward(const dsa_group_args* a, dsa_index_handle* h
                                     void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Top-k for callers that cannot allocate device memory.  (The pages have no counterpart:
+ * this is a deployment convenience of this library, not a step of the method.)
+ *
+ * Same selection and output as dsa_topk (same arguments minus the workspace), computed by
+ * the multi-CTA segmented variant with its scratch in a fixed array inside the library
+ * (DSA_TOPK_NO_ALLOC_SCRATCH_BYTES of device memory, held by every GPU that loads the
+ * library until the process exits).  For callers whose device memory is wholly owned by
+ * another allocator (e.g. an engine that reserves the whole KV pool up front) or that must
+ * not call cudaMalloc / cudaFree, whose implicit device-wide synchronisation would stall
+ * other streams.  Nothing is allocated on any call.
+ *   - n_rows <= DSA_TOPK_NO_ALLOC_MAX_ROWS, else DSA_ERR_INVALID_ARG (no launch).
+ *   - The first call on each device looks up the array's device address; make that first
+ *     call before any stream capture.
+ *   - All calls share the one array: calls that can overlap on the GPU (different streams,
+ *     or different threads without ordering) race and must be serialised by the caller.
+ *     Each call clears the parts that must start at zero.
+ *   - Rows whose threshold bin holds more than 16,384 candidates take a slower path that
+ *     re-reads the row; the result is the same.
+ */
+#define DSA_TOPK_NO_ALLOC_MAX_ROWS 32
+#define DSA_TOPK_NO_ALLOC_SCRATCH_BYTES (32u * (4096u * 4u + 16u + 16384u * 8u))
+dsa_status dsa_topk_no_alloc(const float* scores, int64_t ld, int32_t n_rows, const int32_t* row_len,
+                             int64_t causal_len0, int64_t max_len, int32_t k, int32_t* idx_out, void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * 78-layer schedule (ailearn "IndexShare：四层共用一次搜索结果"): Full at 0-based layers 0, 1
  * and 2 + 4g; every other layer reuses the closest preceding Full layer.
  */

@@ -25,7 +25,7 @@ EXPORTS = [
     "dsa_sparse_mla_workspace_bytes", "dsa_sparse_mla_attn", "dsa_group_workspace_bytes",
     "indexshare_group_forward", "dsa_layer_is_full", "dsa_layer_producer", "dsa_status_str",
     "dsa_last_error", "dsa_abi_version", "dsa_abi_sizeof", "dsa_sync_status", "dsa_debug_bounded_wait",
-    "dsa_set_wait_limit_ns", "dsa_launch_count",
+    "dsa_set_wait_limit_ns", "dsa_launch_count", "dsa_topk_no_alloc",
 ]
 
 
@@ -88,6 +88,8 @@ def load(path: str = LIB_PATH):
         "dsa_debug_bounded_wait": (S, [c_int64, c_void_p]),
         "dsa_set_wait_limit_ns": (c_int64, [c_int64]),
         "dsa_launch_count": (c_int64, []),
+        "dsa_topk_no_alloc": (S, [c_void_p, c_int64, c_int32, c_void_p, c_int64, c_int64, c_int32, c_void_p,
+                                  c_void_p]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -169,6 +171,16 @@ def topk(scores, k: int, row_len=None, causal_len0: int = 0, max_len=None, out=N
         workspace = torch.empty(need, dtype=torch.uint8, device=scores.device)
     _check(lib.dsa_topk(scores.data_ptr(), scores.stride(0), n, _ptr(row_len), causal_len0, max_len, k,
                         out.data_ptr(), _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream()))
+    return out
+
+
+def topk_no_alloc(scores, k: int, out, row_len=None, causal_len0: int = 0, max_len=None):
+    """a4 for callers that cannot allocate device memory: same result as :func:`topk`, scratch
+    inside the library; `out` [n_rows, k] int32 must be provided (nothing is allocated here)."""
+    n = scores.shape[0]
+    max_len = scores.shape[1] if max_len is None else max_len
+    _check(load().dsa_topk_no_alloc(scores.data_ptr(), scores.stride(0), n, _ptr(row_len), causal_len0, max_len, k,
+                                    out.data_ptr(), _stream()))
     return out
 
 

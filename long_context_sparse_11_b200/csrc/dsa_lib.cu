@@ -700,3 +700,86 @@ dsa_status indexshare_group_forward(const dsa_group_args* a, dsa_index_handle* h
 }
 
 }  // extern "C"
+
+// ================================================================ Top-k without caller scratch
+// The segmented Top-k with its scratch in a fixed device array of this file, for callers that
+// cannot allocate device memory (see dsa_topk_no_alloc in include/dsa.h).
+
+namespace dsa {
+namespace {
+
+constexpr int32_t kNoAllocGcap = 16384;
+constexpr size_t kNoAllocRowHead = static_cast<size_t>(topk::BINS) * 4 + 16;
+static_assert(DSA_TOPK_NO_ALLOC_SCRATCH_BYTES ==
+                  DSA_TOPK_NO_ALLOC_MAX_ROWS * (kNoAllocRowHead + static_cast<size_t>(kNoAllocGcap) * 8),
+              "scratch size and layout disagree");
+static_assert(kNoAllocGcap >= topk::CAND_CAP, "global candidate capacity below the shared one");
+
+// Host code must not use this name as a device address: it is looked up per device below.
+static __device__ __align__(256) uint8_t g_topk_scratch[DSA_TOPK_NO_ALLOC_SCRATCH_BYTES];
+
+uint8_t* g_topk_scratch_addr[64] = {};
+std::mutex g_topk_scratch_mu;
+
+// Once per device, with that device current: the array's device address.
+dsa_status topk_scratch_address(uint8_t** out) {
+  int dev = 0;
+  DSA_TRY(cuda_check(cudaGetDevice(&dev), "cudaGetDevice"));
+  if (dev < 0 || dev >= 64) return fail(DSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_topk_scratch_mu);
+  if (!g_topk_scratch_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_topk_scratch);
+    if (e != cudaSuccess || !p) return cuda_check(e, "cudaGetSymbolAddress(top-k scratch)");
+    g_topk_scratch_addr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = g_topk_scratch_addr[dev];
+  return DSA_OK;
+}
+
+}  // namespace
+}  // namespace dsa
+
+extern "C" dsa_status dsa_topk_no_alloc(const float* scores, int64_t ld, int32_t n_rows, const int32_t* row_len,
+                                        int64_t causal_len0, int64_t max_len, int32_t k, int32_t* idx_out,
+                                        void* stream) {
+  if (k < 1 || k > DSA_MAX_K) return fail(DSA_ERR_INVALID_ARG, "k %d not in [1,2048]", k);
+  if (n_rows < 0 || ld <= 0 || ld % 4 || max_len < 0 || ld > INT32_MAX)
+    return fail(DSA_ERR_INVALID_ARG, "bad n_rows / ld / max_len");
+  if (n_rows > DSA_TOPK_NO_ALLOC_MAX_ROWS)
+    return fail(DSA_ERR_INVALID_ARG,
+                "dsa_topk_no_alloc takes at most %d rows (fixed scratch of %u bytes), got %d; "
+                "use dsa_topk with a workspace",
+                DSA_TOPK_NO_ALLOC_MAX_ROWS, DSA_TOPK_NO_ALLOC_SCRATCH_BYTES, n_rows);
+  if (n_rows == 0) return DSA_OK;
+  if (!scores || !aligned16(scores) || !idx_out || !aligned16(idx_out))
+    return fail(DSA_ERR_INVALID_ARG, "scores / idx_out null or misaligned");
+  if (!row_len && causal_len0 < 0) return fail(DSA_ERR_INVALID_ARG, "causal_len0 < 0");
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  uint8_t* scratch = nullptr;
+  DSA_TRY(topk_scratch_address(&scratch));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t cap = std::min(ld, max_len);
+  const int64_t by_len = std::max<int64_t>(1, (cap + 8191) / 8192);
+  const int64_t segs = std::max<int64_t>(1, std::min<int64_t>((4LL * ds->sms + n_rows - 1) / n_rows, by_len));
+  const int32_t seg_len = static_cast<int32_t>(std::max<int64_t>(4, align_up(static_cast<size_t>((cap + segs - 1) / segs), 4)));
+  topk::SegWs sw;
+  sw.hist = reinterpret_cast<uint32_t*>(scratch);
+  sw.counters = reinterpret_cast<int32_t*>(scratch + static_cast<size_t>(n_rows) * topk::BINS * 4);
+  const size_t head = static_cast<size_t>(n_rows) * kNoAllocRowHead;
+  sw.cand_key = reinterpret_cast<uint32_t*>(scratch + head);
+  sw.cand_idx = reinterpret_cast<int32_t*>(scratch + head + static_cast<size_t>(n_rows) * kNoAllocGcap * 4);
+  sw.gcap = kNoAllocGcap;
+  // the histograms and counters of the previous call must not leak into this one
+  DSA_TRY(cuda_check(cudaMemsetAsync(scratch, 0, head, st), "clear top-k scratch"));
+  dim3 grid(static_cast<unsigned>(segs), static_cast<unsigned>(n_rows));
+  topk::topk_seg_hist_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k, seg_len,
+                                                                 sw);
+  topk::topk_seg_filter_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k,
+                                                                   seg_len, sw, idx_out);
+  topk::topk_seg_resolve_kernel<<<n_rows, topk::THREADS, sizeof(topk::Smem), st>>>(scores, ld, row_len, causal_len0,
+                                                                                  cap, k, sw, idx_out);
+  count_launch(3);
+  return cuda_check(cudaGetLastError(), "no-alloc top-k launch");
+}
