@@ -73,13 +73,20 @@ def barrier(ws):
 
 
 def max_over_ranks(x, ws):
+    """Max of a per-rank timer over all ranks (the job's time is its slowest rank)."""
     if ws == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(tokens_per_rank, steps, ws, total_ms_max):
+    """Whole-job tokens/s: every rank processes its own group per step (weak scaling)."""
+    return tokens_per_rank * ws * steps / (total_ms_max / 1e3)
 
 
 # ----------------------------------------------------------------------------- workload
@@ -331,7 +338,7 @@ def run_ours(args, ws, rank, local):
     dsa.sync_status()
     total_ms = max_over_ranks(sum(t_steps), ws)
     ms_per_step = total_ms / args.steps
-    value = counts["tokens"] * ws / (total_ms / 1e3) * args.steps
+    value = job_throughput(counts["tokens"], args.steps, ws, total_ms)
     clocks = clk.summary()
 
     hbm, bf16_peak, peak_kind = measured_peaks()

@@ -306,9 +306,11 @@ dsa_status launch_topk(const float* scores, int64_t ld, int32_t n_rows, const in
 }
 
 int32_t mla_splits(int32_t n_q, int32_t k, int sms) {
+  // persistent CTAs take (row, split) items round-robin: aim for >= 2 items per SM when the
+  // rows alone are too few, with equal tiles per split
   const int32_t tiles = (k + mla::TILE - 1) / mla::TILE;
-  if (n_q >= sms || tiles <= 1) return 1;
-  int32_t s = (sms + n_q - 1) / n_q;
+  if (n_q >= 2 * sms || tiles <= 1) return 1;
+  int32_t s = (2 * sms + n_q - 1) / n_q;
   s = std::min(s, tiles);
   // balance: equal tiles per split
   const int32_t tps = (tiles + s - 1) / s;
@@ -355,7 +357,8 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
     p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
                                          static_cast<size_t>(n_q) * p.n_split * 64 * 512 * 4);
   }
-  const unsigned grid = static_cast<unsigned>(n_q) * p.n_split;
+  const unsigned grid = static_cast<unsigned>(
+      std::min<int64_t>(static_cast<int64_t>(n_q) * p.n_split, static_cast<int64_t>(ds->sms)));
   if (paged)
     mla::sparse_mla_kernel<true><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
   else

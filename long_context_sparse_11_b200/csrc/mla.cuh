@@ -5,23 +5,31 @@
 // 64 x 512 fp32 output fits in 256 TMEM columns:
 //   S^T[key, head]  = KV[key, 0:576] . Q[head, 0:576]        M = 128 keys,  N = 64 heads
 //   O^T[dim, head] += V^T[dim, key]  . P^T[key, head]        M = 128 dims (x4), N = 64 heads
-// S^T puts one key on each TMEM lane, so the softmax thread of lane t owns key t: masking,
-// per-key FP8 dequant scales and the P^T row are all thread-local; only the per-head max
-// and sum cross lanes (shuffle transpose-reduce + 4-warp shared-memory step).  The running
-// max is updated lazily (only when a head's max grows by more than 2^8), so O^T is
-// rescaled in TMEM rarely.
+// S^T puts one key on each TMEM lane, so masking, the per-key FP8 scale and the P^T row are
+// thread-local to the softmax thread of that lane; only the per-head max and sum cross lanes
+// (shuffle transpose-reduce + a shared-memory step over the 4 lane quadrants).  The running
+// max is updated lazily (only when a head's max grows by more than 2^8), so O^T is rarely
+// rescaled in TMEM.
 //
 // Shared memory: Q as 9 K-major 64-dim sub-tiles [64 heads x 128 B] (72 KB) and one
-// 128-key KV tile as 9 sub-tiles [128 keys x 128 B] (144 KB), all 128-byte swizzled.
-// The same KV bytes are the K-major A operand of S^T and the MN-major A operand (V^T) of
-// O^T.  Once S^T of a tile has completed, its RoPE sub-tile (dims 512..575) is free and
-// receives P^T [128 keys x 64 heads], the MN-major B operand of the second MMA.
+// 128-key KV tile as 9 sub-tiles [128 keys x 128 B] (144 KB), 128-byte swizzled.  The same
+// KV bytes are the K-major A operand of S^T and the MN-major A operand (V^T) of O^T; once
+// S^T has completed, the RoPE sub-tile (dims 512..575) receives P^T [128 keys x 64 heads],
+// the MN-major B operand of the second MMA.
 //
-// Rows are gathered with 16-byte cp.async (bf16 cache) or 16-byte loads + e4m3 -> f16
-// conversion (paged FP8 cache; the MMAs then run kind::f16 on f16 operands, exact for
-// e4m3 values, and the per-token scale is applied to the logits and folded into P^T).
+// Pipelining with one KV tile: every sub-tile has its own "full" barrier and every pair of
+// sub-tiles (one 128-dim block of V) its own "empty" barrier, committed when the PV MMAs of
+// that block complete.  The gather of tile j+1 therefore streams into the sub-tiles that
+// PV(j) has finished with while PV(j) still runs on the others, and S^T(j+1) starts as soon
+// as its first sub-tile lands.  CTAs are persistent over (query row, key split) items.
 //
-// Warps 0-3: softmax / output; warps 4-7: gather; warp 8: TMEM owner + MMA issuer.
+// Rows are gathered with 16-byte cp.async, several sub-tiles in flight per thread (bf16
+// cache), or 16-byte loads + e4m3 -> f16 conversion (paged FP8 cache; the MMAs then run
+// kind::f16 on f16 operands, exact for e4m3 values; the per-token scale is applied to the
+// logits and folded into P^T).
+//
+// Warps 0-7: softmax / output (warp w: lane quadrant w%4, heads 32*(w/4) .. +31);
+// warps 8-15: gather; warp 16: TMEM owner + MMA issuer.
 #pragma once
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -39,19 +47,26 @@ constexpr int OFF_KV = NSUB * SUB_Q;
 constexpr int OFF_P = OFF_KV + 8 * SUB_KV;  // RoPE sub-tile, reused for P^T
 constexpr int OFF_MISC = OFF_KV + NSUB * SUB_KV;
 // misc layout (bytes from OFF_MISC)
-constexpr int M_BAR = 0;          // 6 mbarriers
-constexpr int M_TMEM = 64;
-constexpr int M_ABORT = 68;
-constexpr int M_FLAG = 72;
-constexpr int M_MRUN = 128;       // float[64]
+constexpr int N_BARS = 18;
+constexpr int M_TMEM = N_BARS * 8;
+constexpr int M_ABORT = M_TMEM + 4;
+constexpr int M_FLAG = M_TMEM + 8;
+constexpr int M_MRUN = 256;          // float[64], log2 units
 constexpr int M_ALPHA = M_MRUN + 256;
 constexpr int M_LTOT = M_ALPHA + 256;
-constexpr int M_RED = M_LTOT + 256;  // float[4][64]
+constexpr int M_RED = M_LTOT + 256;  // float[4 quadrants][64 heads]
 constexpr int MISC_BYTES = M_RED + 1024;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
-constexpr int THREADS = 288;
+constexpr int SM_WARPS = 8, GA_WARPS = 8;
+constexpr int SM_THREADS = SM_WARPS * 32, GA_THREADS = GA_WARPS * 32;
+constexpr int MMA_WARP = SM_WARPS + GA_WARPS;
+constexpr int THREADS = (MMA_WARP + 1) * 32;
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t TM_S = 256;  // S^T buffers at columns 256, 320
+constexpr int LAG = 4;          // sub-tiles in flight per gather thread before it signals
+
+// barrier indices
+constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 3, B_PVDONE = 4, B_FULL = 5, B_EMPTY = 14;
 
 struct Params {
   const uint16_t* q;         // [n_q,64,576] bf16
@@ -77,21 +92,21 @@ struct Params {
   uint64_t wait_ns;
 };
 
-// Max (or sum) over the 32 lanes of a warp for 64 per-lane values; lane l ends with the
-// results for heads 2l and 2l+1.
+// Max (or sum) over the 32 lanes of a warp for 32 per-lane values; lane l ends with the
+// result for value index l.
 template <bool MAX>
-__device__ __forceinline__ float2 warp_reduce64(const float (&v)[64], int lane) {
-  float a[32];
+__device__ __forceinline__ float warp_reduce32(const float (&v)[32], int lane) {
+  float a[16];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < 16; ++i) {
     const bool hi = lane & 16;
-    const float keep = hi ? v[32 + i] : v[i];
-    const float give = hi ? v[i] : v[32 + i];
+    const float keep = hi ? v[16 + i] : v[i];
+    const float give = hi ? v[i] : v[16 + i];
     const float o = __shfl_xor_sync(0xffffffffu, give, 16);
     a[i] = MAX ? fmaxf(keep, o) : keep + o;
   }
 #pragma unroll
-  for (int w = 32, bit = 8; w >= 4; w >>= 1, bit >>= 1) {
+  for (int w = 16, bit = 8; w >= 2; w >>= 1, bit >>= 1) {
 #pragma unroll
     for (int i = 0; i < w / 2; ++i) {
       const bool hi = lane & bit;
@@ -101,7 +116,7 @@ __device__ __forceinline__ float2 warp_reduce64(const float (&v)[64], int lane) 
       a[i] = MAX ? fmaxf(keep, o) : keep + o;
     }
   }
-  return make_float2(a[0], a[1]);
+  return a[0];
 }
 
 // Physical cache row of idx value v of sequence seq, or -1 when v is not a valid token.
@@ -129,6 +144,46 @@ __device__ __forceinline__ int64_t kv_row(const Params& p, int32_t seq, int32_t 
   return static_cast<int64_t>(pg) * 64 + (v & 63);
 }
 
+// Work item -> (query row, idx row, first tile, number of tiles).
+struct Item {
+  int32_t row, irow, j0, n_tiles, split;
+};
+__device__ __forceinline__ Item make_item(const Params& p, int32_t item) {
+  Item it;
+  it.row = item / p.n_split;
+  it.split = item % p.n_split;
+  it.irow = it.row / p.rows_per_idx;
+  const int32_t all = (p.k + TILE - 1) / TILE;
+  const int32_t tps = (all + p.n_split - 1) / p.n_split;
+  it.j0 = it.split * tps;
+  it.n_tiles = max(0, min(it.j0 + tps, all) - it.j0);
+  return it;
+}
+
+__device__ __forceinline__ uint32_t pack_pair(float a, float b, bool f16) {
+  if (f16) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// e4m3 x16 (one 16-byte chunk) -> two 16-byte chunks of f16 (exact).
+__device__ __forceinline__ void e4m3x16_to_f16(uint4 raw, uint4& o0, uint4& o1) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t r[8];
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[q4] & 0xFFFFu), __NV_E4M3);
+    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[q4] >> 16), __NV_E4M3);
+    r[2 * q4] = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
+    r[2 * q4 + 1] = static_cast<uint32_t>(b.x) | (static_cast<uint32_t>(b.y) << 16);
+  }
+  o0 = make_uint4(r[0], r[1], r[2], r[3]);
+  o1 = make_uint4(r[4], r[5], r[6], r[7]);
+}
+
 template <bool PAGED>
 __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -136,8 +191,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw_addr);
   uint8_t* misc = smem + OFF_MISC;
-  const uint32_t bar = base + OFF_MISC + M_BAR;
-  const uint32_t q_full = bar, kv_full = bar + 8, s_full = bar + 16, p_full = bar + 24, kv_empty = bar + 32;
+  const uint32_t bar0 = base + OFF_MISC;
+  auto bar = [&](int i) { return bar0 + 8u * i; };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + M_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + M_ABORT);
   volatile int* rescale_flag = reinterpret_cast<volatile int*>(misc + M_FLAG);
@@ -145,322 +200,351 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
   float* alpha = reinterpret_cast<float*>(misc + M_ALPHA);
   float* l_tot = reinterpret_cast<float*>(misc + M_LTOT);
   float* red = reinterpret_cast<float*>(misc + M_RED);
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int32_t row = blockIdx.x / p.n_split;
-  const int32_t split = blockIdx.x % p.n_split;
-  const int32_t irow = row / p.rows_per_idx;  // idx row == sequence in paged mode
-  const int32_t* idx_row = p.idx + static_cast<int64_t>(irow) * p.k;
-  const int32_t n_tiles_all = (p.k + TILE - 1) / TILE;
-  const int32_t tps = (n_tiles_all + p.n_split - 1) / p.n_split;
-  const int32_t j0 = split * tps;
-  const int32_t j1 = min(j0 + tps, n_tiles_all);
-  const int32_t n_tiles = max(j1 - j0, 0);
-  const int32_t seq_len = PAGED ? p.seq_lens[irow] : 0;
+  const int32_t n_items = p.n_q * p.n_split;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 128);
-    mbar_init(kv_full, 128);
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(kv_empty, 1);
+    mbar_init(bar(B_QFULL), GA_THREADS);
+    mbar_init(bar(B_QEMPTY), 1);
+    mbar_init(bar(B_SFULL), 1);
+    mbar_init(bar(B_PFULL), SM_THREADS);
+    mbar_init(bar(B_PVDONE), 1);
+    for (int d = 0; d < NSUB; ++d) mbar_init(bar(B_FULL + d), GA_THREADS);
+    for (int g = 0; g < 4; ++g) mbar_init(bar(B_EMPTY + g), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x < 64) m_run[threadIdx.x] = -INFINITY;
-  if (warp == 8) tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+  if (warp == MMA_WARP) tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------------ gather warps
-    const int gt = threadIdx.x - 128;
-    const int gw = warp - 4;
-    // Q row -> 9 K-major sub-tiles (bf16 copy, or bf16 -> f16 for the FP8 cache path)
-    const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q + static_cast<int64_t>(row) * 64 * 576);
-    for (int c = gt; c < 64 * 72; c += 128) {
-      const int h = c / 72, ch = c % 72;
-      const uint32_t dst = base + OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7);
-      if (!PAGED) {
-        cp_async16(dst, qsrc + h * 1152 + ch * 16, 16);
-      } else {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qsrc + h * 1152 + ch * 16));
-        uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-        uint4 o;
-        uint32_t* ov = &o.x;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
-          const __half2 hh = __floats2half2_rn(lo, hi);
-          ov[i] = *reinterpret_cast<const uint32_t*>(&hh);
-        }
-        *reinterpret_cast<uint4*>(smem + (dst - base)) = o;
-      }
-    }
-    if (!PAGED) cp_async_wait_all();
-    fence_async_smem();
-    mbar_arrive(q_full);
-
-    for (int i = 0; i < n_tiles; ++i) {
-      const int j = j0 + i;
-      if (!mbar_wait(kv_empty, (i & 1) ^ 1, abort_flag, p.status, p.wait_ns)) break;
-      const int key0 = gw * 32;
-      const int32_t jj = j * TILE + key0 + lane;
-      const int32_t v = jj < p.k ? idx_row[jj] : -1;
-      const int64_t prow = kv_row<PAGED>(p, irow, v, seq_len);
-      for (int kk = 0; kk < 32; ++kk) {
-        const int key = key0 + kk;
-        const int64_t r = __shfl_sync(0xffffffffu, prow, kk);
+  if (warp >= SM_WARPS && warp < MMA_WARP) {
+    // ================================================================= gather warps
+    const int gt_ = threadIdx.x - SM_THREADS;  // 0..255
+    const int gw = warp - SM_WARPS;
+    uint32_t gtile = 0;
+    bool ok = true;
+    for (int32_t item = blockIdx.x, it_n = 0; item < n_items && ok; item += gridDim.x, ++it_n) {
+      const Item it = make_item(p, item);
+      const int32_t seq_len = PAGED ? p.seq_lens[it.irow] : 0;
+      const int32_t* idx_row = p.idx + static_cast<int64_t>(it.irow) * p.k;
+      // ---- query row -> 9 K-major sub-tiles (bf16 copy, or bf16 -> f16 for the FP8 cache path)
+      if (!mbar_wait(bar(B_QEMPTY), (it_n & 1) ^ 1, abort_flag, p.status, p.wait_ns)) break;
+      const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q + static_cast<int64_t>(it.row) * 64 * 576);
+      for (int c = gt_; c < 64 * 72; c += GA_THREADS) {
+        const int h = c / 72, ch = c % 72;
+        const uint32_t off = OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7);
         if (!PAGED) {
-          const uint8_t* src = p.kv + (r >= 0 ? r : 0) * p.row_stride * 2;
-#pragma unroll
-          for (int t = 0; t < 3; ++t) {
-            const int ch = lane + 32 * t;
-            if (ch < 72) {
-              const uint32_t dst = base + OFF_KV + (ch >> 3) * SUB_KV + sw128_off(key, ch & 7);
-              cp_async16(dst, src + ch * 16, r >= 0 ? 16 : 0);
-            }
-          }
+          cp_async16(base + off, qsrc + h * 1152 + ch * 16, 16);
         } else {
-          const uint8_t* src = p.kv + (r >= 0 ? r : 0) * 576;
+          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qsrc + h * 1152 + ch * 16));
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t o[4];
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int ch = lane + 32 * t;  // 16 e4m3 values = dims [16ch, 16ch+16)
-            if (ch < 36) {
-              uint4 raw = make_uint4(0, 0, 0, 0);
-              if (r >= 0) raw = __ldg(reinterpret_cast<const uint4*>(src + ch * 16));
-              uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-              uint4 o0, o1;
-              uint32_t* ov0 = &o0.x;
-              uint32_t* ov1 = &o1.x;
-#pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) {
-                const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(
-                    static_cast<__nv_fp8x2_storage_t>(w[q4] & 0xFFFFu), __NV_E4M3);
-                const __half2_raw bb = __nv_cvt_fp8x2_to_halfraw2(
-                    static_cast<__nv_fp8x2_storage_t>(w[q4] >> 16), __NV_E4M3);
-                const uint32_t pa = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
-                const uint32_t pb = static_cast<uint32_t>(bb.x) | (static_cast<uint32_t>(bb.y) << 16);
-                if (q4 < 2) {
-                  ov0[2 * q4] = pa;
-                  ov0[2 * q4 + 1] = pb;
-                } else {
-                  ov1[2 * (q4 - 2)] = pa;
-                  ov1[2 * (q4 - 2) + 1] = pb;
-                }
-              }
-              const int sub = ch >> 2, c8 = 2 * (ch & 3);
-              *reinterpret_cast<uint4*>(smem + OFF_KV + sub * SUB_KV + sw128_off(key, c8)) = o0;
-              *reinterpret_cast<uint4*>(smem + OFF_KV + sub * SUB_KV + sw128_off(key, c8 + 1)) = o1;
-            }
-          }
+          for (int i = 0; i < 4; ++i)
+            o[i] = pack_pair(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u), true);
+          *reinterpret_cast<uint4*>(smem + off) = make_uint4(o[0], o[1], o[2], o[3]);
         }
       }
       if (!PAGED) cp_async_wait_all();
       fence_async_smem();
-      mbar_arrive(kv_full);
+      mbar_arrive(bar(B_QFULL));
+      // ---- KV tiles
+      for (int32_t t = 0; t < it.n_tiles && ok; ++t, ++gtile) {
+        const int32_t j = it.j0 + t;
+        const uint32_t par = (gtile & 1) ^ 1;
+        if (!PAGED) {
+          // thread covers chunk (lane & 7) of keys 32i + 4*gw + (lane >> 3), i = 0..3
+          const int chunk = lane & 7;
+          const uint8_t* src[4];
+          uint32_t nbytes[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int key = 32 * i + 4 * gw + (lane >> 3);
+            const int32_t jj = j * TILE + key;
+            const int32_t v = jj < p.k ? idx_row[jj] : -1;
+            const int64_t r = kv_row<false>(p, it.irow, v, seq_len);
+            src[i] = p.kv + (r >= 0 ? r : 0) * p.row_stride * 2 + chunk * 16;
+            nbytes[i] = r >= 0 ? 16u : 0u;
+          }
+          for (int d = 0; d < NSUB; ++d) {
+            if ((d & 1) == 0) {
+              const int g = d < 8 ? d / 2 : -1;
+              const int b = g >= 0 ? B_EMPTY + g : B_PVDONE;
+              if (!mbar_wait(bar(b), par, abort_flag, p.status, p.wait_ns)) {
+                ok = false;
+                break;
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int key = 32 * i + 4 * gw + (lane >> 3);
+              cp_async16(base + OFF_KV + d * SUB_KV + sw128_off(key, chunk), src[i] + d * 128, nbytes[i]);
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            if (d >= LAG) {
+              asm volatile("cp.async.wait_group %0;" ::"n"(LAG) : "memory");
+              fence_async_smem();
+              mbar_arrive(bar(B_FULL + d - LAG));
+            }
+          }
+          if (!ok) break;
+          cp_async_wait_all();
+          fence_async_smem();
+          for (int d = NSUB - LAG; d < NSUB; ++d) mbar_arrive(bar(B_FULL + d));
+        } else {
+          // thread covers 16 fp8 values (part = lane & 3) of keys 64r + 8*gw + (lane >> 2), r = 0, 1
+          const int part = lane & 3;
+          const uint8_t* src[2];
+          bool valid[2];
+#pragma unroll
+          for (int r2 = 0; r2 < 2; ++r2) {
+            const int key = 64 * r2 + 8 * gw + (lane >> 2);
+            const int32_t jj = j * TILE + key;
+            const int32_t v = jj < p.k ? idx_row[jj] : -1;
+            const int64_t r = kv_row<true>(p, it.irow, v, seq_len);
+            valid[r2] = r >= 0;
+            src[r2] = p.kv + (r >= 0 ? r : 0) * 576 + part * 16;
+          }
+          for (int d = 0; d < NSUB; ++d) {
+            if ((d & 1) == 0) {
+              const int g = d < 8 ? d / 2 : -1;
+              const int b = g >= 0 ? B_EMPTY + g : B_PVDONE;
+              if (!mbar_wait(bar(b), par, abort_flag, p.status, p.wait_ns)) {
+                ok = false;
+                break;
+              }
+            }
+            uint4 raw[2];
+#pragma unroll
+            for (int r2 = 0; r2 < 2; ++r2)
+              raw[r2] = valid[r2] ? __ldg(reinterpret_cast<const uint4*>(src[r2] + d * 64)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int r2 = 0; r2 < 2; ++r2) {
+              const int key = 64 * r2 + 8 * gw + (lane >> 2);
+              uint4 o0, o1;
+              e4m3x16_to_f16(raw[r2], o0, o1);
+              *reinterpret_cast<uint4*>(smem + OFF_KV + d * SUB_KV + sw128_off(key, 2 * part)) = o0;
+              *reinterpret_cast<uint4*>(smem + OFF_KV + d * SUB_KV + sw128_off(key, 2 * part + 1)) = o1;
+            }
+            fence_async_smem();
+            mbar_arrive(bar(B_FULL + d));
+          }
+        }
+      }
     }
-  } else if (warp == 8) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == MMA_WARP) {
+    // ================================================================= MMA issuer
     if (lane == 0) {
       constexpr uint32_t FMT = PAGED ? 0u : 1u;  // f16 operands for the FP8 cache, else bf16
       constexpr uint32_t ID_S = make_idesc(FMT, FMT, 0, 0, 128, 64);
       constexpr uint32_t ID_PV = make_idesc(FMT, FMT, 1, 1, 128, 64);
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status, p.wait_ns);
-      tc_fence_after();
-      for (int i = 0; i < n_tiles && ok; ++i) {
-        if (!mbar_wait(kv_full, i & 1, abort_flag, p.status, p.wait_ns)) break;
+      uint32_t gtile = 0;
+      bool ok = true;
+      for (int32_t item = blockIdx.x, it_n = 0; item < n_items && ok; item += gridDim.x, ++it_n) {
+        const Item it = make_item(p, item);
+        if (!mbar_wait(bar(B_QFULL), it_n & 1, abort_flag, p.status, p.wait_ns)) break;
         tc_fence_after();
-        const uint32_t ds = tmem + TM_S + 64u * (i & 1);
-#pragma unroll 1
-        for (int d = 0; d < NSUB; ++d) {
+        if (it.n_tiles == 0) mma_commit(bar(B_QEMPTY));
+        for (int32_t t = 0; t < it.n_tiles && ok; ++t, ++gtile) {
+          const uint32_t par = gtile & 1;
+          const uint32_t ds = tmem + TM_S + 64u * par;
+          for (int d = 0; d < NSUB; ++d) {
+            if (!mbar_wait(bar(B_FULL + d), par, abort_flag, p.status, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t a = make_sdesc(base + OFF_KV + d * SUB_KV + kk * 32, 16, 1024);
-            const uint64_t b = make_sdesc(base + OFF_Q + d * SUB_Q + kk * 32, 16, 1024);
-            mma_f16(ds, a, b, ID_S, (d | kk) != 0);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t a = make_sdesc(base + OFF_KV + d * SUB_KV + kk * 32, 16, 1024);
+              const uint64_t b = make_sdesc(base + OFF_Q + d * SUB_Q + kk * 32, 16, 1024);
+              mma_f16(ds, a, b, ID_S, (d | kk) != 0);
+            }
           }
-        }
-        mma_commit(s_full);
-        if (!mbar_wait(p_full, i & 1, abort_flag, p.status, p.wait_ns)) break;
-        tc_fence_after();
+          if (!ok) break;
+          mma_commit(bar(B_SFULL));
+          if (t == it.n_tiles - 1) mma_commit(bar(B_QEMPTY));
+          if (!mbar_wait(bar(B_PFULL), par, abort_flag, p.status, p.wait_ns)) break;
+          tc_fence_after();
 #pragma unroll 1
-        for (int mb = 0; mb < 4; ++mb) {
+          for (int mb = 0; mb < 4; ++mb) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = make_sdesc(base + OFF_KV + 2 * mb * SUB_KV + kk * 2048, SUB_KV, 1024);
-            const uint64_t b = make_sdesc(base + OFF_P + kk * 2048, SUB_KV, 1024);
-            mma_f16(tmem + 64u * mb, a, b, ID_PV, (i > 0 || kk > 0));
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t a = make_sdesc(base + OFF_KV + 2 * mb * SUB_KV + kk * 2048, SUB_KV, 1024);
+              const uint64_t b = make_sdesc(base + OFF_P + kk * 2048, SUB_KV, 1024);
+              mma_f16(tmem + 64u * mb, a, b, ID_PV, (t > 0 || kk > 0));
+            }
+            mma_commit(bar(B_EMPTY + mb));
           }
+          mma_commit(bar(B_PVDONE));
         }
-        mma_commit(kv_empty);
       }
     }
   } else {
-    // ------------------------------------------------------------------ softmax warps 0-3
-    const int t = threadIdx.x;  // TMEM lane = key within tile (S^T) = dim within block (O^T)
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    float lsum[64];
-#pragma unroll
-    for (int h = 0; h < 64; ++h) lsum[h] = 0.f;
+    // ================================================================= softmax / output warps 0-7
+    const int quad = warp & 3, hh = warp >> 2;
+    const int key = quad * 32 + lane;                 // TMEM lane: key of S^T, dim of an O^T block
+    const int st = warp * 32 + lane;                  // 0..255
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t hcol = 32u * hh;
+    uint32_t gtile = 0;
     bool ok = true;
-    for (int i = 0; i < n_tiles && ok; ++i) {
-      const int j = j0 + i;
-      const int32_t jj = j * TILE + t;
-      const int32_t v = jj < p.k ? idx_row[jj] : -1;
-      const int64_t prow = kv_row<PAGED>(p, irow, v, seq_len);
-      const bool valid = prow >= 0;
-      const float kscale = PAGED ? (valid ? p.kv_scale[prow] : 0.f) : 1.f;
-      if (!mbar_wait(s_full, i & 1, abort_flag, p.status, p.wait_ns)) break;
-      tc_fence_after();
-      float z[64];
-      {
-        uint32_t x[32];
-        const uint32_t ta = tmem + TM_S + 64u * (i & 1) + lane_off;
-        DSA_TMEM_LD_X32(ta, x);
+    for (int32_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const Item it = make_item(p, item);
+      const int32_t seq_len = PAGED ? p.seq_lens[it.irow] : 0;
+      const int32_t* idx_row = p.idx + static_cast<int64_t>(it.irow) * p.k;
+      if (quad == 0) m_run[hcol + lane] = -INFINITY;
+      named_bar(1, SM_THREADS);
+      float lsum[32];
 #pragma unroll
-        for (int h = 0; h < 32; ++h) z[h] = __uint_as_float(x[h]);
-        DSA_TMEM_LD_X32(ta + 32, x);
-#pragma unroll
-        for (int h = 0; h < 32; ++h) z[32 + h] = __uint_as_float(x[h]);
-      }
-      const float zs = p.scale_log2 * kscale;
-#pragma unroll
-      for (int h = 0; h < 64; ++h) z[h] = valid ? z[h] * zs : -INFINITY;
-      const float2 wm = warp_reduce64<true>(z, lane);
-      red[warp * 64 + 2 * lane] = wm.x;
-      red[warp * 64 + 2 * lane + 1] = wm.y;
-      if (t == 0) *rescale_flag = 0;
-      named_bar(1, 128);
-      if (t < 64) {
-        const float tmax = fmaxf(fmaxf(red[t], red[64 + t]), fmaxf(red[128 + t], red[192 + t]));
-        const float mo = m_run[t];
-        float a = 1.f;
-        if (tmax > -INFINITY && (mo == -INFINITY || tmax > mo + 8.f)) {
-          a = (mo == -INFINITY) ? 0.f : exp2f(mo - tmax);
-          m_run[t] = tmax;
-          *rescale_flag = 1;
+      for (int h = 0; h < 32; ++h) lsum[h] = 0.f;
+      for (int32_t t = 0; t < it.n_tiles; ++t, ++gtile) {
+        const uint32_t par = gtile & 1;
+        const int32_t jj = (it.j0 + t) * TILE + key;
+        const int32_t v = jj < p.k ? idx_row[jj] : -1;
+        const int64_t prow = kv_row<PAGED>(p, it.irow, v, seq_len);
+        const bool valid = prow >= 0;
+        const float kscale = PAGED ? (valid ? p.kv_scale[prow] : 0.f) : 1.f;
+        if (!mbar_wait(bar(B_SFULL), par, abort_flag, p.status, p.wait_ns)) {
+          ok = false;
+          break;
         }
-        alpha[t] = a;
-      }
-      named_bar(1, 128);
-      const bool resc = *rescale_flag != 0;
-      // probabilities, partial row sums, P^T row
-      uint32_t pk[32];
-#pragma unroll
-      for (int h2 = 0; h2 < 32; ++h2) {
-        float pv[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int h = 2 * h2 + e;
-          const float m = m_run[h];
-          const float pr = valid ? exp2f(z[h] - (m == -INFINITY ? 0.f : m)) : 0.f;
-          lsum[h] = resc ? fmaf(lsum[h], alpha[h], pr) : lsum[h] + pr;
-          pv[e] = pr * kscale;
-        }
-        if (PAGED) {
-          const __half2 hh = __floats2half2_rn(pv[0], pv[1]);
-          pk[h2] = *reinterpret_cast<const uint32_t*>(&hh);
-        } else {
-          const __nv_bfloat162 bb = __floats2bfloat162_rn(pv[0], pv[1]);
-          pk[h2] = *reinterpret_cast<const uint32_t*>(&bb);
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(smem + OFF_P + sw128_off(t, c)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      if (resc && i > 0) {
-        // O^T (dims on lanes, heads on columns) *= alpha[head]; PV of the previous tile is done
-        if (!mbar_wait(kv_empty, (i - 1) & 1, abort_flag, p.status, p.wait_ns)) break;
         tc_fence_after();
-#pragma unroll 1
-        for (int mb = 0; mb < 4; ++mb) {
+        float z[32];
+        {
+          uint32_t x[32];
+          DSA_TMEM_LD_X32(tmem + TM_S + 64u * par + hcol + lane_off, x);
+          const float zs = p.scale_log2 * kscale;
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
+          for (int h = 0; h < 32; ++h) z[h] = valid ? __uint_as_float(x[h]) * zs : -INFINITY;
+        }
+        red[quad * 64 + hcol + lane] = warp_reduce32<true>(z, lane);
+        if (st == 0) *rescale_flag = 0;
+        named_bar(1, SM_THREADS);
+        if (quad == 0) {
+          const int h = hcol + lane;
+          const float tmax = fmaxf(fmaxf(red[h], red[64 + h]), fmaxf(red[128 + h], red[192 + h]));
+          const float mo = m_run[h];
+          float a = 1.f;
+          if (tmax > -INFINITY && (mo == -INFINITY || tmax > mo + 8.f)) {
+            a = (mo == -INFINITY) ? 0.f : exp2f(mo - tmax);
+            m_run[h] = tmax;
+            *rescale_flag = 1;
+          }
+          alpha[h] = a;
+        }
+        named_bar(1, SM_THREADS);
+        const bool resc = *rescale_flag != 0;
+        uint32_t pk[16];
+#pragma unroll
+        for (int h2 = 0; h2 < 16; ++h2) {
+          float pv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int h = 2 * h2 + e;
+            const float m = m_run[hcol + h];
+            const float pr = valid ? exp2f(z[h] - (m == -INFINITY ? 0.f : m)) : 0.f;
+            lsum[h] = resc ? fmaf(lsum[h], alpha[hcol + h], pr) : lsum[h] + pr;
+            pv[e] = pr * kscale;
+          }
+          pk[h2] = pack_pair(pv[0], pv[1], PAGED);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(smem + OFF_P + sw128_off(key, 4 * hh + c)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        if (resc && t > 0) {
+          // O^T (dims on lanes, heads on columns) *= alpha; PV of the previous tile is done
+          if (!mbar_wait(bar(B_PVDONE), par ^ 1, abort_flag, p.status, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int mb = 0; mb < 4; ++mb) {
             uint32_t x[32];
-            const uint32_t ta = tmem + 64u * mb + 32u * hh + lane_off;
+            const uint32_t ta = tmem + 64u * mb + hcol + lane_off;
             DSA_TMEM_LD_X32(ta, x);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) x[c] = __float_as_uint(__uint_as_float(x[c]) * alpha[32 * hh + c]);
+            for (int c = 0; c < 32; ++c) x[c] = __float_as_uint(__uint_as_float(x[c]) * alpha[hcol + c]);
             DSA_TMEM_ST_X32(ta, x);
           }
         }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(B_PFULL));
       }
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full);
-    }
-    // ---- final: wait for the last PV, reduce row sums, write the output
-    if (n_tiles > 0) ok = mbar_wait(kv_empty, (n_tiles - 1) & 1, abort_flag, p.status, p.wait_ns);
-    tc_fence_after();
-    const float2 ws = warp_reduce64<false>(lsum, lane);
-    named_bar(1, 128);
-    red[warp * 64 + 2 * lane] = ws.x;
-    red[warp * 64 + 2 * lane + 1] = ws.y;
-    named_bar(1, 128);
-    if (t < 64) l_tot[t] = red[t] + red[64 + t] + red[128 + t] + red[192 + t];
-    named_bar(1, 128);
-    if (ok && !*abort_flag) {
+      if (!ok) break;
+      // ---- end of item: wait for the last PV, reduce row sums, write the output
+      if (it.n_tiles > 0) {
+        if (!mbar_wait(bar(B_PVDONE), (gtile - 1) & 1, abort_flag, p.status, p.wait_ns)) break;
+        tc_fence_after();
+      }
+      red[quad * 64 + hcol + lane] = warp_reduce32<false>(lsum, lane);
+      named_bar(1, SM_THREADS);
+      if (quad == 0) {
+        const int h = hcol + lane;
+        l_tot[h] = red[h] + red[64 + h] + red[128 + h] + red[192 + h];
+      }
+      named_bar(1, SM_THREADS);
       if (p.n_split == 1) {
-        uint16_t* orow = p.out + static_cast<int64_t>(row) * 64 * 512;
+        uint16_t* orow = p.out + static_cast<int64_t>(it.row) * 64 * 512;
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
-#pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t x[32];
-            if (n_tiles > 0) {
-              DSA_TMEM_LD_X32(tmem + 64u * mb + 32u * hh + lane_off, x);
-            } else {
+          uint32_t x[32];
+          if (it.n_tiles > 0) {
+            DSA_TMEM_LD_X32(tmem + 64u * mb + hcol + lane_off, x);
+          } else {
 #pragma unroll
-              for (int c = 0; c < 32; ++c) x[c] = 0u;
-            }
+            for (int c = 0; c < 32; ++c) x[c] = 0u;
+          }
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const int h = 32 * hh + c;
-              const float l = l_tot[h];
-              const float o = l > 0.f ? __uint_as_float(x[c]) / l : 0.f;
-              const __nv_bfloat16 ob = __float2bfloat16_rn(o);
-              orow[h * 512 + mb * 128 + t] = *reinterpret_cast<const uint16_t*>(&ob);
-            }
+          for (int c = 0; c < 32; ++c) {
+            const int h = hcol + c;
+            const float l = l_tot[h];
+            const float o = l > 0.f ? __uint_as_float(x[c]) / l : 0.f;
+            const __nv_bfloat16 ob = __float2bfloat16_rn(o);
+            orow[h * 512 + mb * 128 + key] = *reinterpret_cast<const uint16_t*>(&ob);
           }
         }
-        if (p.lse && t < 64) {
-          const float l = l_tot[t];
-          p.lse[static_cast<int64_t>(row) * 64 + t] =
-              l > 0.f ? (m_run[t] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (p.lse && quad == 0) {
+          const int h = hcol + lane;
+          const float l = l_tot[h];
+          p.lse[static_cast<int64_t>(it.row) * 64 + h] =
+              l > 0.f ? (m_run[h] + log2f(l)) * 0.69314718055994531f : -INFINITY;
         }
       } else {
-        const int64_t pr = static_cast<int64_t>(row) * p.n_split + split;
+        const int64_t pr = static_cast<int64_t>(it.row) * p.n_split + it.split;
         float* po = p.part_o + pr * 64 * 512;
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
-#pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t x[32];
-            if (n_tiles > 0) {
-              DSA_TMEM_LD_X32(tmem + 64u * mb + 32u * hh + lane_off, x);
-            } else {
+          uint32_t x[32];
+          if (it.n_tiles > 0) {
+            DSA_TMEM_LD_X32(tmem + 64u * mb + hcol + lane_off, x);
+          } else {
 #pragma unroll
-              for (int c = 0; c < 32; ++c) x[c] = 0u;
-            }
-#pragma unroll
-            for (int c = 0; c < 32; ++c) po[(32 * hh + c) * 512 + mb * 128 + t] = __uint_as_float(x[c]);
+            for (int c = 0; c < 32; ++c) x[c] = 0u;
           }
+#pragma unroll
+          for (int c = 0; c < 32; ++c) po[(hcol + c) * 512 + mb * 128 + key] = __uint_as_float(x[c]);
         }
-        if (t < 64) {
-          p.part_ml[pr * 128 + t] = m_run[t];
-          p.part_ml[pr * 128 + 64 + t] = l_tot[t];
+        if (quad == 0) {
+          const int h = hcol + lane;
+          p.part_ml[pr * 128 + h] = m_run[h];
+          p.part_ml[pr * 128 + 64 + h] = l_tot[h];
         }
       }
+      tc_fence_before();
+      named_bar(1, SM_THREADS);  // m_run / l_tot / red are reused by the next item
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 8) tmem_dealloc(tmem, TMEM_COLS);
+  if (warp == MMA_WARP) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 // Combine split-KV partials: one CTA of 128 threads per (row, head), 4 dims per thread.
