@@ -261,22 +261,19 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
           break;
         }
         tc_fence_after();
-#pragma unroll 1
-        for (int j = 0; j < QPW; ++j) {
-          const int qq = PAGED ? 0 : half * QPW + j;  // query within the group
-          uint32_t x[32];
-          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + bf * C::N + qq * 32;
-          DSA_TMEM_LD_X32(taddr, x);
+        // head sum of one query from registers: ReLU, per-head weight, packed FMA on head pairs
+        auto score = [&](const uint32_t (&x)[32], int qq) {
           const float4* wv = reinterpret_cast<const float4*>(w_s + (g * C::NQ + qq) * 32);
-          float acc = 0.f;
+          float a0 = 0.f, a1 = 0.f;
 #pragma unroll
           for (int h4 = 0; h4 < 8; ++h4) {
             const float4 ww = wv[h4];
-            acc = fmaf(ww.x, fmaxf(__uint_as_float(x[4 * h4 + 0]), 0.f), acc);
-            acc = fmaf(ww.y, fmaxf(__uint_as_float(x[4 * h4 + 1]), 0.f), acc);
-            acc = fmaf(ww.z, fmaxf(__uint_as_float(x[4 * h4 + 2]), 0.f), acc);
-            acc = fmaf(ww.w, fmaxf(__uint_as_float(x[4 * h4 + 3]), 0.f), acc);
+            ffma2(a0, a1, ww.x, ww.y, fmaxf(__uint_as_float(x[4 * h4]), 0.f),
+                  fmaxf(__uint_as_float(x[4 * h4 + 1]), 0.f));
+            ffma2(a0, a1, ww.z, ww.w, fmaxf(__uint_as_float(x[4 * h4 + 2]), 0.f),
+                  fmaxf(__uint_as_float(x[4 * h4 + 3]), 0.f));
           }
+          float acc = a0 + a1;
           if (FP8) acc *= sk;
           if (PAGED) {
             if (s_abs < len) p.scores[static_cast<int64_t>(b) * p.ld + s_abs] = acc;
@@ -284,6 +281,22 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
             const int32_t row = r0 + g * C::NQ + qq;
             if (row < p.n_q && s_abs <= static_cast<int64_t>(p.q_pos0) + row && s_abs < p.n_tokens)
               p.scores[static_cast<int64_t>(row) * p.ld + s_abs] = acc;
+          }
+        };
+        const uint32_t trow = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + bf * C::N;
+        const int q0 = PAGED ? 0 : half * QPW;
+        // TMEM loads run one query ahead of the math
+        uint32_t xa[32], xb[32];
+        DSA_TMEM_LD_X32_NOWAIT(trow + q0 * 32, xa);
+#pragma unroll
+        for (int j = 0; j < QPW; j += 2) {
+          DSA_TMEM_WAIT_LD(xa);
+          if (j + 1 < QPW) DSA_TMEM_LD_X32_NOWAIT(trow + (q0 + j + 1) * 32, xb);
+          score(xa, q0 + j);
+          if (j + 1 < QPW) {
+            DSA_TMEM_WAIT_LD(xb);
+            if (j + 2 < QPW) DSA_TMEM_LD_X32_NOWAIT(trow + (q0 + j + 2) * 32, xa);
+            score(xb, q0 + j + 1);
           }
         }
         tc_fence_before();

@@ -28,8 +28,9 @@
 // kind::f16 on f16 operands, exact for e4m3 values; the per-token scale is applied to the
 // logits and folded into P^T).
 //
-// Warps 0-7: softmax / output (warp w: lane quadrant w%4, heads 32*(w/4) .. +31);
-// warps 8-15: gather; warp 16: TMEM owner + MMA issuer.
+// Warps 0-7: softmax / output (warp w: lane quadrant w%4, heads 32*(w/4) .. +31), and part of
+// the next tile's gather; warps 8-14: query rows and the rest of the gather; warp 15: TMEM
+// owner + MMA issuer.  16 warps = 4 per SM sub-partition, so each thread may use 128 registers.
 #pragma once
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -50,15 +51,16 @@ constexpr int OFF_MISC = OFF_KV + NSUB * SUB_KV;
 constexpr int N_BARS = 18;
 constexpr int M_TMEM = N_BARS * 8;
 constexpr int M_ABORT = M_TMEM + 4;
-constexpr int M_FLAG = M_TMEM + 8;
+constexpr int M_NEED = M_TMEM + 8;   // int[2]: "a head's max moved" flag per tile parity
 constexpr int M_MRUN = 256;          // float[64], log2 units
 constexpr int M_ALPHA = M_MRUN + 256;
 constexpr int M_LTOT = M_ALPHA + 256;
 constexpr int M_RED = M_LTOT + 256;  // float[4 quadrants][64 heads]
 constexpr int MISC_BYTES = M_RED + 1024;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
-constexpr int SM_WARPS = 8, GA_WARPS = 8;
+constexpr int SM_WARPS = 8, GA_WARPS = 7;  // 16 warps: 4 per SM sub-partition, 128 registers each
 constexpr int SM_THREADS = SM_WARPS * 32, GA_THREADS = GA_WARPS * 32;
+constexpr int NG = SM_THREADS + GA_THREADS;  // threads that gather KV rows (softmax warps help)
 constexpr int MMA_WARP = SM_WARPS + GA_WARPS;
 constexpr int THREADS = (MMA_WARP + 1) * 32;
 constexpr int TMEM_COLS = 512;
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
   auto bar = [&](int i) { return bar0 + 8u * i; };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(misc + M_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + M_ABORT);
-  volatile int* rescale_flag = reinterpret_cast<volatile int*>(misc + M_FLAG);
+  volatile int* need_flags = reinterpret_cast<volatile int*>(misc + M_NEED);
   float* m_run = reinterpret_cast<float*>(misc + M_MRUN);
   float* alpha = reinterpret_cast<float*>(misc + M_ALPHA);
   float* l_tot = reinterpret_cast<float*>(misc + M_LTOT);
@@ -209,9 +211,11 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
     mbar_init(bar(B_SFULL), 1);
     mbar_init(bar(B_PFULL), SM_THREADS);
     mbar_init(bar(B_PVDONE), 1);
-    for (int d = 0; d < NSUB; ++d) mbar_init(bar(B_FULL + d), GA_THREADS);
+    for (int d = 0; d < NSUB; ++d) mbar_init(bar(B_FULL + d), NG);
     for (int g = 0; g < 4; ++g) mbar_init(bar(B_EMPTY + g), 1);
     *abort_flag = 0;
+    need_flags[0] = 0;
+    need_flags[1] = 0;
     fence_mbar_init();
   }
   if (warp == MMA_WARP) tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
@@ -220,20 +224,107 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  // One thread's share (g in [0, NG)) of KV tile t of item `it` (global tile counter gtile):
+  // 16-byte chunks c = g, g + NG, ... of every 64-dim sub-tile, chunk c = (key c/8, 16 bytes
+  // c%8) for the bf16 cache, or (key c/4, 16 e4m3 values c%4) for the paged FP8 cache.
+  // Sub-tiles are written in order, each pair once PV of the previous tile has released it;
+  // "full" arrivals lag by up to LAG sub-tiles and are flushed before any blocking wait.
+  auto gather_tile = [&](const Item& it, int32_t t, uint32_t gtile, int g) -> bool {
+    const int32_t j = it.j0 + t;
+    const uint32_t par = (gtile & 1) ^ 1;
+    const int32_t seq_len = PAGED ? p.seq_lens[it.irow] : 0;
+    const int32_t* idx_row = p.idx + static_cast<int64_t>(it.irow) * p.k;
+    if (!PAGED) {
+      constexpr int MAXC = (1024 + NG - 1) / NG;
+      const uint8_t* src[MAXC];
+      uint32_t nb[MAXC], dst[MAXC];
+#pragma unroll
+      for (int i = 0; i < MAXC; ++i) {
+        const int c = g + i * NG;
+        const int key = c >> 3, chunk = c & 7;
+        int64_t r = -1;
+        if (c < 1024) {
+          const int32_t jj = j * TILE + key;
+          const int32_t v = jj < p.k ? idx_row[jj] : -1;
+          r = kv_row<false>(p, it.irow, v, seq_len);
+        }
+        src[i] = p.kv + (r >= 0 ? r : 0) * p.row_stride * 2 + chunk * 16;
+        nb[i] = r >= 0 ? 16u : 0u;
+        dst[i] = c < 1024 ? sw128_off(key, chunk) : 0xFFFFFFFFu;
+      }
+      int pending = 0;
+      for (int d = 0; d < NSUB; ++d) {
+        if ((d & 1) == 0) {
+          const uint32_t eb = bar(d < 8 ? B_EMPTY + d / 2 : B_PVDONE);
+          if (!mbar_try_wait(eb, par)) {
+            if (pending) {
+              cp_async_wait_all();
+              fence_async_smem();
+              for (int q = d - pending; q < d; ++q) mbar_arrive(bar(B_FULL + q));
+              pending = 0;
+            }
+            if (!mbar_wait(eb, par, abort_flag, p.status, p.wait_ns)) return false;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < MAXC; ++i)
+          if (dst[i] != 0xFFFFFFFFu) cp_async16(base + OFF_KV + d * SUB_KV + dst[i], src[i] + d * 128, nb[i]);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if (++pending > LAG) {
+          asm volatile("cp.async.wait_group %0;" ::"n"(LAG) : "memory");
+          fence_async_smem();
+          mbar_arrive(bar(B_FULL + d - LAG));
+          pending = LAG;
+        }
+      }
+      cp_async_wait_all();
+      fence_async_smem();
+      for (int q = NSUB - pending; q < NSUB; ++q) mbar_arrive(bar(B_FULL + q));
+    } else {
+      // parts c = g, g + NG of the 128 keys x 4 parts; each part: 16 e4m3 values of every sub-tile,
+      // all 9 loaded up front (loads do not touch shared memory, so they need no release)
+      for (int c = g; c < 512; c += NG) {
+        const int key = c >> 2, part = c & 3;
+        const int32_t jj = j * TILE + key;
+        const int32_t v = jj < p.k ? idx_row[jj] : -1;
+        const int64_t r = kv_row<true>(p, it.irow, v, seq_len);
+        const uint8_t* src = p.kv + (r >= 0 ? r : 0) * 576 + part * 16;
+        uint4 raw[NSUB];
+#pragma unroll
+        for (int d = 0; d < NSUB; ++d)
+          raw[d] = r >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + d * 64)) : make_uint4(0, 0, 0, 0);
+        const bool last = c + NG >= 512;  // this thread's last part: signal the sub-tiles after it
+#pragma unroll
+        for (int d = 0; d < NSUB; ++d) {
+          if ((d & 1) == 0) {
+            if (!mbar_wait(bar(d < 8 ? B_EMPTY + d / 2 : B_PVDONE), par, abort_flag, p.status, p.wait_ns))
+              return false;
+          }
+          uint4 o0, o1;
+          e4m3x16_to_f16(raw[d], o0, o1);
+          *reinterpret_cast<uint4*>(smem + OFF_KV + d * SUB_KV + sw128_off(key, 2 * part)) = o0;
+          *reinterpret_cast<uint4*>(smem + OFF_KV + d * SUB_KV + sw128_off(key, 2 * part + 1)) = o1;
+          if (last) {
+            fence_async_smem();
+            mbar_arrive(bar(B_FULL + d));
+          }
+        }
+      }
+    }
+    return true;
+  };
+
   if (warp >= SM_WARPS && warp < MMA_WARP) {
     // ================================================================= gather warps
-    const int gt_ = threadIdx.x - SM_THREADS;  // 0..255
-    const int gw = warp - SM_WARPS;
+    const int gq = threadIdx.x - SM_THREADS;  // query-row loader index
     uint32_t gtile = 0;
     bool ok = true;
     for (int32_t item = blockIdx.x, it_n = 0; item < n_items && ok; item += gridDim.x, ++it_n) {
       const Item it = make_item(p, item);
-      const int32_t seq_len = PAGED ? p.seq_lens[it.irow] : 0;
-      const int32_t* idx_row = p.idx + static_cast<int64_t>(it.irow) * p.k;
       // ---- query row -> 9 K-major sub-tiles (bf16 copy, or bf16 -> f16 for the FP8 cache path)
       if (!mbar_wait(bar(B_QEMPTY), (it_n & 1) ^ 1, abort_flag, p.status, p.wait_ns)) break;
       const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q + static_cast<int64_t>(it.row) * 64 * 576);
-      for (int c = gt_; c < 64 * 72; c += GA_THREADS) {
+      for (int c = gq; c < 64 * 72; c += GA_THREADS) {
         const int h = c / 72, ch = c % 72;
         const uint32_t off = OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7);
         if (!PAGED) {
@@ -251,89 +342,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
       if (!PAGED) cp_async_wait_all();
       fence_async_smem();
       mbar_arrive(bar(B_QFULL));
-      // ---- KV tiles
-      for (int32_t t = 0; t < it.n_tiles && ok; ++t, ++gtile) {
-        const int32_t j = it.j0 + t;
-        const uint32_t par = (gtile & 1) ^ 1;
-        if (!PAGED) {
-          // thread covers chunk (lane & 7) of keys 32i + 4*gw + (lane >> 3), i = 0..3
-          const int chunk = lane & 7;
-          const uint8_t* src[4];
-          uint32_t nbytes[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int key = 32 * i + 4 * gw + (lane >> 3);
-            const int32_t jj = j * TILE + key;
-            const int32_t v = jj < p.k ? idx_row[jj] : -1;
-            const int64_t r = kv_row<false>(p, it.irow, v, seq_len);
-            src[i] = p.kv + (r >= 0 ? r : 0) * p.row_stride * 2 + chunk * 16;
-            nbytes[i] = r >= 0 ? 16u : 0u;
-          }
-          for (int d = 0; d < NSUB; ++d) {
-            if ((d & 1) == 0) {
-              const int g = d < 8 ? d / 2 : -1;
-              const int b = g >= 0 ? B_EMPTY + g : B_PVDONE;
-              if (!mbar_wait(bar(b), par, abort_flag, p.status, p.wait_ns)) {
-                ok = false;
-                break;
-              }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int key = 32 * i + 4 * gw + (lane >> 3);
-              cp_async16(base + OFF_KV + d * SUB_KV + sw128_off(key, chunk), src[i] + d * 128, nbytes[i]);
-            }
-            asm volatile("cp.async.commit_group;" ::: "memory");
-            if (d >= LAG) {
-              asm volatile("cp.async.wait_group %0;" ::"n"(LAG) : "memory");
-              fence_async_smem();
-              mbar_arrive(bar(B_FULL + d - LAG));
-            }
-          }
-          if (!ok) break;
-          cp_async_wait_all();
-          fence_async_smem();
-          for (int d = NSUB - LAG; d < NSUB; ++d) mbar_arrive(bar(B_FULL + d));
-        } else {
-          // thread covers 16 fp8 values (part = lane & 3) of keys 64r + 8*gw + (lane >> 2), r = 0, 1
-          const int part = lane & 3;
-          const uint8_t* src[2];
-          bool valid[2];
-#pragma unroll
-          for (int r2 = 0; r2 < 2; ++r2) {
-            const int key = 64 * r2 + 8 * gw + (lane >> 2);
-            const int32_t jj = j * TILE + key;
-            const int32_t v = jj < p.k ? idx_row[jj] : -1;
-            const int64_t r = kv_row<true>(p, it.irow, v, seq_len);
-            valid[r2] = r >= 0;
-            src[r2] = p.kv + (r >= 0 ? r : 0) * 576 + part * 16;
-          }
-          for (int d = 0; d < NSUB; ++d) {
-            if ((d & 1) == 0) {
-              const int g = d < 8 ? d / 2 : -1;
-              const int b = g >= 0 ? B_EMPTY + g : B_PVDONE;
-              if (!mbar_wait(bar(b), par, abort_flag, p.status, p.wait_ns)) {
-                ok = false;
-                break;
-              }
-            }
-            uint4 raw[2];
-#pragma unroll
-            for (int r2 = 0; r2 < 2; ++r2)
-              raw[r2] = valid[r2] ? __ldg(reinterpret_cast<const uint4*>(src[r2] + d * 64)) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int r2 = 0; r2 < 2; ++r2) {
-              const int key = 64 * r2 + 8 * gw + (lane >> 2);
-              uint4 o0, o1;
-              e4m3x16_to_f16(raw[r2], o0, o1);
-              *reinterpret_cast<uint4*>(smem + OFF_KV + d * SUB_KV + sw128_off(key, 2 * part)) = o0;
-              *reinterpret_cast<uint4*>(smem + OFF_KV + d * SUB_KV + sw128_off(key, 2 * part + 1)) = o1;
-            }
-            fence_async_smem();
-            mbar_arrive(bar(B_FULL + d));
-          }
-        }
-      }
+      for (int32_t t = 0; t < it.n_tiles && ok; ++t, ++gtile) ok = gather_tile(it, t, gtile, threadIdx.x);
     }
   } else if (warp == MMA_WARP) {
     // ================================================================= MMA issuer
@@ -398,6 +407,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
       const int32_t* idx_row = p.idx + static_cast<int64_t>(it.irow) * p.k;
       if (quad == 0) m_run[hcol + lane] = -INFINITY;
       named_bar(1, SM_THREADS);
+      if (it.n_tiles > 0 && !gather_tile(it, 0, gtile, threadIdx.x)) break;
       float lsum[32];
 #pragma unroll
       for (int h = 0; h < 32; ++h) lsum[h] = 0.f;
@@ -421,41 +431,65 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
 #pragma unroll
           for (int h = 0; h < 32; ++h) z[h] = valid ? __uint_as_float(x[h]) * zs : -INFINITY;
         }
-        red[quad * 64 + hcol + lane] = warp_reduce32<true>(z, lane);
-        if (st == 0) *rescale_flag = 0;
-        named_bar(1, SM_THREADS);
-        if (quad == 0) {
-          const int h = hcol + lane;
-          const float tmax = fmaxf(fmaxf(red[h], red[64 + h]), fmaxf(red[128 + h], red[192 + h]));
-          const float mo = m_run[h];
-          float a = 1.f;
-          if (tmax > -INFINITY && (mo == -INFINITY || tmax > mo + 8.f)) {
-            a = (mo == -INFINITY) ? 0.f : exp2f(mo - tmax);
-            m_run[h] = tmax;
-            *rescale_flag = 1;
-          }
-          alpha[h] = a;
+        // Lazy running max: the cross-lane reduction is needed only when some logit exceeds
+        // its head's running max by more than 8 (log2 units) -- always on an item's first tile.
+        volatile int* need = need_flags + (gtile & 1);
+        bool exceed = false;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float4 m4 = *reinterpret_cast<const float4*>(m_run + hcol + 4 * c);
+          exceed |= (z[4 * c] > m4.x + 8.f) | (z[4 * c + 1] > m4.y + 8.f) | (z[4 * c + 2] > m4.z + 8.f) |
+                    (z[4 * c + 3] > m4.w + 8.f);
         }
+        if (__any_sync(0xffffffffu, exceed) && lane == 0) *need = 1;
         named_bar(1, SM_THREADS);
-        const bool resc = *rescale_flag != 0;
-        uint32_t pk[16];
-#pragma unroll
-        for (int h2 = 0; h2 < 16; ++h2) {
-          float pv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int h = 2 * h2 + e;
-            const float m = m_run[hcol + h];
-            const float pr = valid ? exp2f(z[h] - (m == -INFINITY ? 0.f : m)) : 0.f;
-            lsum[h] = resc ? fmaf(lsum[h], alpha[hcol + h], pr) : lsum[h] + pr;
-            pv[e] = pr * kscale;
+        if (st == 0) need_flags[(gtile + 1) & 1] = 0;  // the next tile's flag: its readers are done
+        const bool resc = *need != 0;
+        if (resc) {
+          red[quad * 64 + hcol + lane] = warp_reduce32<true>(z, lane);
+          named_bar(1, SM_THREADS);
+          if (quad == 0) {
+            const int h = hcol + lane;
+            const float tmax = fmaxf(fmaxf(red[h], red[64 + h]), fmaxf(red[128 + h], red[192 + h]));
+            const float mo = m_run[h];
+            float a = 1.f;
+            if (tmax > -INFINITY && (mo == -INFINITY || tmax > mo + 8.f)) {
+              a = (mo == -INFINITY) ? 0.f : ex2_approx(mo - tmax);
+              m_run[h] = tmax;
+            }
+            alpha[h] = a;
           }
-          pk[h2] = pack_pair(pv[0], pv[1], PAGED);
-        }
+          named_bar(1, SM_THREADS);
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(smem + OFF_P + sw128_off(key, 4 * hh + c)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int c = 0; c < 8; ++c) {
+            const float4 a4 = *reinterpret_cast<const float4*>(alpha + hcol + 4 * c);
+            lsum[4 * c] *= a4.x;
+            lsum[4 * c + 1] *= a4.y;
+            lsum[4 * c + 2] *= a4.z;
+            lsum[4 * c + 3] *= a4.w;
+          }
+        }
+        // probabilities 8 heads at a time -> one 16-byte chunk of this key's P^T row
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float m8[8];
+          const float4 ma = *reinterpret_cast<const float4*>(m_run + hcol + 8 * c);
+          const float4 mb = *reinterpret_cast<const float4*>(m_run + hcol + 8 * c + 4);
+          m8[0] = ma.x, m8[1] = ma.y, m8[2] = ma.z, m8[3] = ma.w;
+          m8[4] = mb.x, m8[5] = mb.y, m8[6] = mb.z, m8[7] = mb.w;
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int h = 8 * c + 2 * e;
+            // z = -inf for masked keys, so the probability is exactly 0
+            const float p0 = ex2_approx(z[h] - (m8[2 * e] == -INFINITY ? 0.f : m8[2 * e]));
+            const float p1 = ex2_approx(z[h + 1] - (m8[2 * e + 1] == -INFINITY ? 0.f : m8[2 * e + 1]));
+            lsum[h] += p0;
+            lsum[h + 1] += p1;
+            pk[e] = pack_pair(p0 * kscale, p1 * kscale, PAGED);
+          }
+          *reinterpret_cast<uint4*>(smem + OFF_P + sw128_off(key, 4 * hh + c)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
         if (resc && t > 0) {
           // O^T (dims on lanes, heads on columns) *= alpha; PV of the previous tile is done
           if (!mbar_wait(bar(B_PVDONE), par ^ 1, abort_flag, p.status, p.wait_ns)) {
@@ -476,6 +510,10 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(bar(B_PFULL));
+        if (t + 1 < it.n_tiles && !gather_tile(it, t + 1, gtile + 1, threadIdx.x)) {
+          ok = false;
+          break;
+        }
       }
       if (!ok) break;
       // ---- end of item: wait for the last PV, reduce row sums, write the output

@@ -178,6 +178,44 @@ __host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c) {
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])                      \
       : "memory")
 
+// TMEM load without the wait, and a wait that names the destination registers so that no use
+// of them can be scheduled before it (lets one load overlap the math on the previous one).
+#define DSA_TMEM_LD_X32_NOWAIT(taddr, r)                                                                      \
+  asm volatile(                                                                                               \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17," \
+      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                                      \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),       \
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), \
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),            \
+        "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),            \
+        "=r"(r[30]), "=r"(r[31])                                                                              \
+      : "r"(taddr)                                                                                            \
+      : "memory")
+#define DSA_TMEM_WAIT_LD(r)                                                                                   \
+  asm volatile("tcgen05.wait::ld.sync.aligned;"                                                               \
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),         \
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),      \
+                 "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),   \
+                 "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),   \
+                 "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])                                           \
+               :                                                                                              \
+               : "memory")
+
+// (a0, a1) += (w0, w1) * (x0, x1) as one packed fp32 FMA (fma.rn.f32x2).
+__device__ __forceinline__ void ffma2(float& a0, float& a1, float w0, float w1, float x0, float x1) {
+  asm("{\n\t.reg .b64 A, W, X;\n\tmov.b64 A, {%0, %1};\n\tmov.b64 W, {%2, %3};\n\tmov.b64 X, {%4, %5};\n\t"
+      "fma.rn.f32x2 A, W, X, A;\n\tmov.b64 {%0, %1}, A;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(w0), "f"(w1), "f"(x0), "f"(x1));
+}
+
+// 2^x with the hardware approximation (ex2.approx, flush-to-zero); 2^-inf = 0.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Order-preserving map of fp32 to uint32 (larger float -> larger key); -0 maps like +0.
 __device__ __forceinline__ uint32_t f32_key(float f) {
   uint32_t u = __float_as_uint(f);
