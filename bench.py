@@ -37,7 +37,7 @@ def parse():
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--workload", default="prefill_32k",
-                   choices=["tiny_prefill", "prefill_32k", "prefill_128k_fp8", "decode_b32_mtp4"])
+                   choices=["tiny_prefill", "prefill_32k", "prefill_128k_fp8", "decode_b32_mtp4", "decode_1m_mtp5"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     p.add_argument("--ref-seconds", type=float, default=150.0, help="reference arm total budget")
@@ -99,50 +99,82 @@ def workload_config(name, seq_len=None):
     if seq_len is not None and hasattr(spec, "L"):
         spec = dataclasses.replace(spec, L=seq_len)
     if name.startswith("decode"):
-        return spec, {"workload": name, "batch": spec.batch, "context": f"U[{spec.ctx_lo},{spec.ctx_hi}]",
-                      "rows_per_seq": spec.rows_per_seq, "k": spec.k, "layers_per_group": 4,
-                      "cache": "paged e4m3, 64-token pages", "indexer": "e4m3"}
+        cfg = {"workload": name, "batch": spec.batch, "context": f"U[{spec.ctx_lo},{spec.ctx_hi}]",
+               "rows_per_seq": spec.rows_per_seq, "k": spec.k, "layers": spec.n_layers,
+               "cache": "paged e4m3 (64-token pages), device-resident across steps", "indexer": "e4m3"}
+        if spec.n_layers > 4:
+            cfg["schedule"] = "Full at layers 0, 1, 2+4g; 21 groups per step"
+        return spec, cfg
     return spec, {"workload": name, "seq_len": spec.L, "k": spec.k, "layers_per_group": spec.n_layers,
                   "indexer": "e4m3" if spec.indexer_fp8 else "bf16", "latent_kv": "bf16 [L,576]",
                   "heads": 64, "indexer_heads": 32}
 
 
 def algorithmic_counts(spec, ctx=None):
-    """Algorithmic work of one group: indexer flops, MLA flops per layer, tokens per step."""
+    """Algorithmic work of one group: indexer flops/bytes, MLA flops per layer, query tokens."""
     if hasattr(spec, "L"):
         L, k = spec.L, spec.k
         pairs = L * (L + 1) // 2
         sel = sum(min(k, t + 1) for t in range(L))
         return {"tokens": L, "indexer_flops": 8192.0 * pairs, "mla_flops_per_layer": 139264.0 * sel,
-                "mla_rows": L}
+                "mla_rows": L, "indexer_bytes": None}
     import numpy as np
     ctx = np.asarray(ctx)
     R = spec.rows_per_seq
     sel = float(np.minimum(ctx, spec.k).sum())
     return {"tokens": len(ctx) * R, "indexer_flops": 8192.0 * float(ctx.sum()),
             "mla_flops_per_layer": 139264.0 * sel * R, "mla_rows": len(ctx) * R,
-            "indexer_bytes": 132.0 * float(ctx.sum())}
+            "indexer_bytes": 132.0 * float(ctx.sum()),
+            "mla_bytes_per_layer": sel * 580.0 + len(ctx) * R * 64 * (576 + 512) * 2.0}
 
 
-def build_group(spec, name, dev):
-    """Device inputs and an IndexShareGroup for the workload."""
-    import torch
-    import long_context_sparse_11_b200 as dsa
-    from synth import make_prefill, make_decode
-    if name.startswith("decode"):
-        inp = make_decode(spec, device=dev)
-        ctx_d = torch.from_numpy(inp["ctx"].astype("int32")).to(dev)
-        bt_d = torch.from_numpy(inp["block_table"]).to(dev)
-        keys = dsa.paged_view(inp["idx_keys"], inp["idx_key_scale"], bt_d, ctx_d)
-        kvs = [dsa.paged_view(inp["KV"][l], inp["KV_scale"][l], bt_d, ctx_d) for l in range(4)]
-        g = dsa.IndexShareGroup(inp["q_idx"], inp["w"], keys, spec.k, inp["Q"], kvs, inp["softmax_scale"],
-                                indexer_dtype=dsa.DSA_E4M3, q_rows_per_idx_row=spec.rows_per_seq)
-        return g, inp
-    inp = make_prefill(spec, device=dev)
-    g = dsa.IndexShareGroup(inp["q_idx"], inp["w"], dsa.dense_view(inp["k_idx"]), spec.k, inp["Q"],
-                            [dsa.dense_view(x) for x in inp["KV"]], inp["softmax_scale"],
-                            indexer_dtype=dsa.DSA_E4M3 if spec.indexer_fp8 else dsa.DSA_BF16)
-    return g, inp
+class Workload:
+    """Device inputs and the IndexShare groups of one step (1 group, or 21 for 78 layers)."""
+
+    def __init__(self, spec, name, dev):
+        import torch
+        import long_context_sparse_11_b200 as dsa
+        from synth import make_prefill, make_decode, make_decode_indexer
+        self.name, self.spec = name, spec
+        self.groups, self.step_inputs, self.layers_per_group = [], [], []
+        if name.startswith("decode"):
+            inp = make_decode(spec, device=dev)
+            self.inp = inp
+            ctx_d = torch.from_numpy(inp["ctx"].astype("int32")).to(dev)
+            bt_d = torch.from_numpy(inp["block_table"]).to(dev)
+            kvs = [dsa.paged_view(inp["KV"][l], inp["KV_scale"][l], bt_d, ctx_d) for l in range(spec.n_layers)]
+            fulls = [l for l in range(spec.n_layers) if dsa.layer_is_full(l)] if spec.n_layers > 4 else [0]
+            ends = fulls[1:] + [spec.n_layers]
+            for f, e in zip(fulls, ends):
+                ind = inp if f == 0 else make_decode_indexer(spec, f, inp["n_pages"], len(inp["ctx"]), dev)
+                keys = dsa.paged_view(ind["idx_keys"], ind["idx_key_scale"], bt_d, ctx_d)
+                g = dsa.IndexShareGroup(ind["q_idx"], ind["w"], keys, spec.k, inp["Q"][f:e], kvs[f:e],
+                                        inp["softmax_scale"], indexer_dtype=dsa.DSA_E4M3,
+                                        q_rows_per_idx_row=spec.rows_per_seq, first_layer=f)
+                self.groups.append(g)
+                self.layers_per_group.append(e - f)
+                # a decode step's new inputs: the indexer query and weights, the MLA query rows
+                self.step_inputs += [ind["q_idx"], ind["w"]] + list(inp["Q"][f:e])
+            self.counts = algorithmic_counts(spec, inp["ctx"])
+        else:
+            inp = make_prefill(spec, device=dev)
+            self.inp = inp
+            g = dsa.IndexShareGroup(inp["q_idx"], inp["w"], dsa.dense_view(inp["k_idx"]), spec.k, inp["Q"],
+                                    [dsa.dense_view(x) for x in inp["KV"]], inp["softmax_scale"],
+                                    indexer_dtype=dsa.DSA_E4M3 if spec.indexer_fp8 else dsa.DSA_BF16)
+            self.groups.append(g)
+            self.layers_per_group.append(spec.n_layers)
+            # a prefill step's inputs: everything the group reads
+            self.step_inputs = [inp["q_idx"], inp["w"], inp["k_idx"]] + list(inp["Q"]) + list(inp["KV"])
+            self.counts = algorithmic_counts(spec)
+
+    @property
+    def outputs(self):
+        return [t for g in self.groups for t in g.out + g.lse]
+
+    def forward(self):
+        for g in self.groups:
+            g.forward()
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -226,18 +258,20 @@ def oracle_rows_per_second(spec, name, inp, budget_s, seed_rows=0):
         return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
     if name.startswith("decode"):
+        nl = 4 if len(inp["Q"]) <= 4 else 1   # the first IndexShare group (layers 0..3, or layer 0 of 78)
         host = {"ctx": inp["ctx"], "block_table": inp["block_table"], "k": spec.k, "rows_per_seq": spec.rows_per_seq,
                 "softmax_scale": spec.softmax_scale, "q_idx": host_bits(inp["q_idx"]), "w": inp["w"].cpu().numpy(),
                 "idx_keys": inp["idx_keys"].cpu().numpy(), "idx_key_scale": inp["idx_key_scale"].cpu().numpy(),
-                "Q": [host_bits(q) for q in inp["Q"]], "KV": [x.cpu().numpy() for x in inp["KV"]],
-                "KV_scale": [x.cpu().numpy() for x in inp["KV_scale"]]}
+                "Q": [host_bits(q) for q in inp["Q"][:nl]], "KV": [x.cpu().numpy() for x in inp["KV"][:nl]],
+                "KV_scale": [x.cpu().numpy() for x in inp["KV_scale"][:nl]]}
         order = list(np.random.default_rng(seed_rows).permutation(len(inp["ctx"])))
         done, t0 = 0, time.perf_counter()
         while order and time.perf_counter() - t0 < budget_s:
             O.group_decode(host, seqs=[order.pop()])
             done += spec.rows_per_seq
         el = time.perf_counter() - t0
-        return done / el, f"{done // spec.rows_per_seq} whole sequences (all {spec.rows_per_seq} rows, 4 layers)", el
+        return done / el, (f"{done // spec.rows_per_seq} whole sequences (all {spec.rows_per_seq} rows, indexer, "
+                           f"Top-k and {nl} layer(s) of the first group)"), el
     L = spec.L
     host = {"L": L, "k": spec.k, "softmax_scale": spec.softmax_scale, "k_idx": host_bits(inp["k_idx"]),
             "q_idx": _LazyRows(inp["q_idx"]), "w": _LazyRows(inp["w"], bf16=False),
@@ -284,6 +318,7 @@ def cpu_cores():
 
 
 def run_ours(args, ws, rank, local):
+    import ctypes
     import torch
     import long_context_sparse_11_b200 as dsa
     from long_context_sparse_11_b200.build import build
@@ -293,25 +328,27 @@ def run_ours(args, ws, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     spec, cfg = workload_config(args.workload, args.seq_len)
-    g, inp = build_group(spec, args.workload, dev)
-    counts = algorithmic_counts(spec, inp.get("ctx"))
+    wl = Workload(spec, args.workload, dev)
+    counts = wl.counts
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.int32, device=dev)   # 1 GiB > 126 MB L2
 
-    # trace events: indexer phase and each layer's sparse MLA launch (recorded once so
-    # that torch creates the underlying CUDA events before their handles are passed on)
-    n_ev = 2 + 2 * 4
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-    for e in evs:
-        e.record(stream)
+    # trace events per group: the Full layer's a1-a4 phase and each layer's sparse MLA launch
+    # (recorded once so that torch creates the CUDA events before their handles are passed on)
+    traces = []
+    for g, nl in zip(wl.groups, wl.layers_per_group):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 + 2 * nl)]
+        for e in evs:
+            e.record(stream)
+        traces.append(evs)
     torch.cuda.synchronize()
-    import ctypes
-    ev_arr = (ctypes.c_void_p * n_ev)(*[e.cuda_event for e in evs])
-    assert all(e.cuda_event for e in evs)
+    arrs = [(ctypes.c_void_p * len(evs))(*[e.cuda_event for e in evs]) for evs in traces]
+    assert all(e.cuda_event for evs in traces for e in evs)
 
     def step(traced):
-        g.args.trace_events = ctypes.cast(ev_arr, ctypes.c_void_p) if traced else None
-        g.forward()
+        for g, arr in zip(wl.groups, arrs):
+            g.args.trace_events = ctypes.cast(arr, ctypes.c_void_p) if traced else None
+        wl.forward()
 
     for _ in range(args.warmup):
         step(False)
@@ -330,60 +367,76 @@ def run_ours(args, ws, rank, local):
             s1.record(stream)
             s1.synchronize()
             t_steps.append(s0.elapsed_time(s1))
-            idx_ms.append(evs[0].elapsed_time(evs[1]))
-            mla_ms.extend(evs[2 + 2 * l].elapsed_time(evs[3 + 2 * l]) for l in range(4))
+            for evs, nl in zip(traces, wl.layers_per_group):
+                idx_ms.append(evs[0].elapsed_time(evs[1]))
+                mla_ms.extend(evs[2 + 2 * l].elapsed_time(evs[3 + 2 * l]) for l in range(nl))
     torch.cuda.synchronize()
     launches = lib.dsa_launch_count() - n0
     barrier(ws)
     dsa.sync_status()
     total_ms = max_over_ranks(sum(t_steps), ws)
     ms_per_step = total_ms / args.steps
-    value = job_throughput(counts["tokens"], args.steps, ws, total_ms)
+    n_groups = len(wl.groups)
+    value = job_throughput(counts["tokens"] * n_groups, args.steps, ws, total_ms)
     clocks = clk.summary()
 
     hbm, bf16_peak, peak_kind = measured_peaks()
     mla_avg = statistics.mean(mla_ms)
-    achieved = counts["mla_flops_per_layer"] / (mla_avg / 1e3) / 1e12
-    roofline = {"kernel": "sparse_mla_kernel (a6)", "bound": "tensor", "achieved": round(achieved, 1),
-                "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(achieved / bf16_peak, 4),
+    idx_avg = statistics.mean(idx_ms)
+    mla_tf = counts["mla_flops_per_layer"] / (mla_avg / 1e3) / 1e12
+    mla_roof = {"kernel": "sparse_mla_kernel (a6)", "bound": "tensor", "achieved": round(mla_tf, 1),
+                "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(mla_tf / bf16_peak, 4),
                 "peak_source": f"{peak_kind} bf16 dense (burst)", "traffic": None,
                 "algorithmic_flops_per_launch": counts["mla_flops_per_layer"], "avg_launch_ms": round(mla_avg, 4)}
-    idx_avg = statistics.mean(idx_ms)
     phases = {"indexer_topk_ms": round(idx_avg, 4), "mla_ms_per_layer": round(mla_avg, 4),
-              "indexer_topk_tflops": round(counts["indexer_flops"] / (idx_avg / 1e3) / 1e12, 1)}
+              "indexer_topk_tflops": round(counts["indexer_flops"] / (idx_avg / 1e3) / 1e12, 1),
+              "groups_per_step": n_groups}
+    roofline = mla_roof
+    if counts.get("indexer_bytes"):
+        gbs = counts["indexer_bytes"] / (idx_avg / 1e3) / 1e9
+        phases["indexer_topk_gbs"] = round(gbs, 1)
+        phases["indexer_topk_hbm_frac"] = round(gbs / hbm, 4)
+        mla_gbs = counts["mla_bytes_per_layer"] / (mla_avg / 1e3) / 1e9
+        phases["mla_gbs"] = round(mla_gbs, 1)
+        if idx_avg * n_groups > mla_avg * sum(wl.layers_per_group):
+            roofline = {"kernel": "indexer_kernel<e4m3,paged> + topk (a2-a4)", "bound": "hbm",
+                        "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                        "peak_source": f"{peak_kind} HBM copy", "traffic": None,
+                        "algorithmic_bytes_per_launch": counts["indexer_bytes"], "avg_launch_ms": round(idx_avg, 4)}
+            phases["mla_roofline"] = mla_roof
+    if n_groups > 1:
+        phases["step_ms_all_layers"] = round(ms_per_step, 4)
 
-    # end to end through the public API: pinned host inputs -> device, group, outputs -> host
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, g, inp, spec, counts, stream, ws)
+        e2e = run_e2e(args, wl, stream, ws)
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline and ws == 1:
-        v, sample, el = oracle_rows_per_second(spec, args.workload, inp, args.cpu_seconds)
+        v, sample, el = oracle_rows_per_second(spec, args.workload, wl.inp, args.cpu_seconds)
         cpu = {"value": round(v, 3), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": sample,
                "seconds": round(el, 1)}
     if rank == 0:
         cfg.update({"l2": "flushed (1 GiB write) between timed steps", "parallelism": f"replicas x{ws}"})
+        dtype = "bf16" if args.workload.startswith("prefill_32k") or args.workload == "tiny_prefill" else "bf16+e4m3"
         line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if not spec.__dict__.get("indexer_fp8")
-                else "bf16+e4m3", "data": "synthetic (seeded SplitMix64 normals)", "config": cfg,
+                "scaling": "weak", "vs_baseline": None, "dtype": dtype,
+                "data": "synthetic (seeded SplitMix64 normals)", "config": cfg,
                 "roofline": roofline, "phases": phases, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
                 "clocks": clocks}
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, g, inp, spec, counts, stream, ws):
+def run_e2e(args, wl, stream, ws):
+    """Same metric through the public API with host buffers: every step copies its inputs from
+    pinned host memory to the device, runs the groups and reads the outputs back."""
     import torch
     import long_context_sparse_11_b200 as dsa
-    dev_in = []
-    for key in ("q_idx", "w", "k_idx", "idx_keys", "idx_key_scale", "Q", "KV", "KV_scale"):
-        v = inp.get(key)
-        for x in (v if isinstance(v, list) else [v]):
-            if hasattr(x, "is_cuda") and x.is_cuda:
-                dev_in.append(x)
+    dev_in = wl.step_inputs
     host_in = [t.cpu().pin_memory() for t in dev_in]
-    host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in g.out + g.lse]
+    outs = wl.outputs
+    host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
     steps = max(2, min(args.steps, 5))
@@ -391,8 +444,8 @@ def run_e2e(args, g, inp, spec, counts, stream, ws):
     def one():
         for h, d in zip(host_in, dev_in):
             d.copy_(h, non_blocking=True)
-        g.forward()
-        for h, d in zip(host_out, g.out + g.lse):
+        wl.forward()
+        for h, d in zip(host_out, outs):
             h.copy_(d, non_blocking=True)
 
     one()
@@ -407,7 +460,8 @@ def run_e2e(args, g, inp, spec, counts, stream, ws):
     e1.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), ws)
     dsa.sync_status()
-    return {"value": round(counts["tokens"] * ws * steps / (ms / 1e3), 1), "unit": UNIT,
+    tokens = wl.counts["tokens"] * len(wl.groups)
+    return {"value": round(tokens * ws * steps / (ms / 1e3), 1), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 3)}
 

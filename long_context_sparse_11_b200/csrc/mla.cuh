@@ -23,8 +23,8 @@
 // PV(j) has finished with while PV(j) still runs on the others, and S^T(j+1) starts as soon
 // as its first sub-tile lands.  CTAs are persistent over (query row, key split) items.
 //
-// Rows are gathered with 16-byte cp.async, several sub-tiles in flight per thread (bf16
-// cache), or 16-byte loads + e4m3 -> f16 conversion (paged FP8 cache; the MMAs then run
+// Rows are gathered with 16-byte cp.async whose completion the hardware reports to the
+// sub-tile's barrier (bf16 cache), or 16-byte loads + e4m3 -> f16 conversion (paged FP8 cache; the MMAs then run
 // kind::f16 on f16 operands, exact for e4m3 values; the per-token scale is applied to the
 // logits and folded into P^T).
 //
@@ -65,7 +65,6 @@ constexpr int MMA_WARP = SM_WARPS + GA_WARPS;
 constexpr int THREADS = (MMA_WARP + 1) * 32;
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t TM_S = 256;  // S^T buffers at columns 256, 320
-constexpr int LAG = 4;          // sub-tiles in flight per gather thread before it signals
 
 // barrier indices
 constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 3, B_PVDONE = 4, B_FULL = 5, B_EMPTY = 14;
@@ -224,82 +223,74 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  // One thread's share (g in [0, NG)) of KV tile t of item `it` (global tile counter gtile):
-  // 16-byte chunks c = g, g + NG, ... of every 64-dim sub-tile, chunk c = (key c/8, 16 bytes
-  // c%8) for the bf16 cache, or (key c/4, 16 e4m3 values c%4) for the paged FP8 cache.
-  // Sub-tiles are written in order, each pair once PV of the previous tile has released it;
-  // "full" arrivals lag by up to LAG sub-tiles and are flushed before any blocking wait.
-  auto gather_tile = [&](const Item& it, int32_t t, uint32_t gtile, int g) -> bool {
+  // One thread's share (g in [0, NG)) of a KV tile: 16-byte chunks c = g, g + NG, ... of every
+  // 64-dim sub-tile, chunk c = (key c/8, 16 bytes c%8) for the bf16 cache, or (key c/4, 16 e4m3
+  // values c%4) for the paged FP8 cache.  `prepare` reads the tile's indices (issued early so
+  // their latency hides behind other work); `issue` writes the sub-tiles in order, each pair
+  // once PV of the previous tile has released it.  bf16: cp.async, and the hardware arrives on
+  // the sub-tile's "full" barrier when this thread's copies have landed (the thread never waits
+  // for them; the MMA issuer fences the async proxy after the barrier).
+  constexpr int MAXC = (1024 + NG - 1) / NG;
+  struct Plan {
+    const uint8_t* src[MAXC];
+    uint32_t nb[MAXC], dst[MAXC];
+  };
+  auto prepare = [&](const Item& it, int32_t t, int g) -> Plan {
+    Plan pl;
     const int32_t j = it.j0 + t;
-    const uint32_t par = (gtile & 1) ^ 1;
     const int32_t seq_len = PAGED ? p.seq_lens[it.irow] : 0;
     const int32_t* idx_row = p.idx + static_cast<int64_t>(it.irow) * p.k;
-    if (!PAGED) {
-      constexpr int MAXC = (1024 + NG - 1) / NG;
-      const uint8_t* src[MAXC];
-      uint32_t nb[MAXC], dst[MAXC];
 #pragma unroll
-      for (int i = 0; i < MAXC; ++i) {
-        const int c = g + i * NG;
-        const int key = c >> 3, chunk = c & 7;
-        int64_t r = -1;
-        if (c < 1024) {
-          const int32_t jj = j * TILE + key;
-          const int32_t v = jj < p.k ? idx_row[jj] : -1;
-          r = kv_row<false>(p, it.irow, v, seq_len);
-        }
-        src[i] = p.kv + (r >= 0 ? r : 0) * p.row_stride * 2 + chunk * 16;
-        nb[i] = r >= 0 ? 16u : 0u;
-        dst[i] = c < 1024 ? sw128_off(key, chunk) : 0xFFFFFFFFu;
-      }
-      int pending = 0;
-      for (int d = 0; d < NSUB; ++d) {
-        if ((d & 1) == 0) {
-          const uint32_t eb = bar(d < 8 ? B_EMPTY + d / 2 : B_PVDONE);
-          if (!mbar_try_wait(eb, par)) {
-            if (pending) {
-              cp_async_wait_all();
-              fence_async_smem();
-              for (int q = d - pending; q < d; ++q) mbar_arrive(bar(B_FULL + q));
-              pending = 0;
-            }
-            if (!mbar_wait(eb, par, abort_flag, p.status, p.wait_ns)) return false;
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < MAXC; ++i)
-          if (dst[i] != 0xFFFFFFFFu) cp_async16(base + OFF_KV + d * SUB_KV + dst[i], src[i] + d * 128, nb[i]);
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        if (++pending > LAG) {
-          asm volatile("cp.async.wait_group %0;" ::"n"(LAG) : "memory");
-          fence_async_smem();
-          mbar_arrive(bar(B_FULL + d - LAG));
-          pending = LAG;
-        }
-      }
-      cp_async_wait_all();
-      fence_async_smem();
-      for (int q = NSUB - pending; q < NSUB; ++q) mbar_arrive(bar(B_FULL + q));
-    } else {
-      // parts c = g, g + NG of the 128 keys x 4 parts; each part: 16 e4m3 values of every sub-tile,
-      // all 9 loaded up front (loads do not touch shared memory, so they need no release)
-      for (int c = g; c < 512; c += NG) {
-        const int key = c >> 2, part = c & 3;
+    for (int i = 0; i < MAXC; ++i) {
+      const int c = g + i * NG;
+      const int key = PAGED ? (c >> 2) : (c >> 3), sub = PAGED ? (c & 3) : (c & 7);
+      const int lim = PAGED ? 512 : 1024;
+      int64_t r = -1;
+      if (c < lim) {
         const int32_t jj = j * TILE + key;
         const int32_t v = jj < p.k ? idx_row[jj] : -1;
-        const int64_t r = kv_row<true>(p, it.irow, v, seq_len);
-        const uint8_t* src = p.kv + (r >= 0 ? r : 0) * 576 + part * 16;
+        r = kv_row<PAGED>(p, it.irow, v, seq_len);
+      }
+      if (PAGED) {
+        pl.src[i] = p.kv + (r >= 0 ? r : 0) * 576 + sub * 16;
+        pl.dst[i] = c < lim ? static_cast<uint32_t>(key * 4 + sub) : 0xFFFFFFFFu;
+      } else {
+        pl.src[i] = p.kv + (r >= 0 ? r : 0) * p.row_stride * 2 + sub * 16;
+        pl.dst[i] = c < lim ? sw128_off(key, sub) : 0xFFFFFFFFu;
+      }
+      pl.nb[i] = r >= 0 ? 16u : 0u;
+    }
+    return pl;
+  };
+  auto issue = [&](const Plan& pl, uint32_t gtile) -> bool {
+    const uint32_t par = (gtile & 1) ^ 1;
+    if (!PAGED) {
+      for (int d = 0; d < NSUB; ++d) {
+        if ((d & 1) == 0 &&
+            !mbar_wait(bar(d < 8 ? B_EMPTY + d / 2 : B_PVDONE), par, abort_flag, p.status, p.wait_ns))
+          return false;
+#pragma unroll
+        for (int i = 0; i < MAXC; ++i)
+          if (pl.dst[i] != 0xFFFFFFFFu)
+            cp_async16(base + OFF_KV + d * SUB_KV + pl.dst[i], pl.src[i] + d * 128, pl.nb[i]);
+        cp_async_arrive_noinc(bar(B_FULL + d));
+      }
+    } else {
+      // each part: 16 e4m3 values of every sub-tile, all 9 loaded before the first wait (loads do
+      // not touch shared memory), converted to f16 and stored once the sub-tile pair is free
+      for (int i = 0; i < MAXC; ++i) {
+        if (pl.dst[i] == 0xFFFFFFFFu) continue;
+        const int key = pl.dst[i] >> 2, part = pl.dst[i] & 3;
         uint4 raw[NSUB];
 #pragma unroll
         for (int d = 0; d < NSUB; ++d)
-          raw[d] = r >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + d * 64)) : make_uint4(0, 0, 0, 0);
-        const bool last = c + NG >= 512;  // this thread's last part: signal the sub-tiles after it
+          raw[d] = pl.nb[i] ? __ldg(reinterpret_cast<const uint4*>(pl.src[i] + d * 64)) : make_uint4(0, 0, 0, 0);
+        const bool last = i + 1 == MAXC || pl.dst[i + 1 < MAXC ? i + 1 : i] == 0xFFFFFFFFu;
 #pragma unroll
         for (int d = 0; d < NSUB; ++d) {
-          if ((d & 1) == 0) {
-            if (!mbar_wait(bar(d < 8 ? B_EMPTY + d / 2 : B_PVDONE), par, abort_flag, p.status, p.wait_ns))
-              return false;
-          }
+          if ((d & 1) == 0 &&
+              !mbar_wait(bar(d < 8 ? B_EMPTY + d / 2 : B_PVDONE), par, abort_flag, p.status, p.wait_ns))
+            return false;
           uint4 o0, o1;
           e4m3x16_to_f16(raw[d], o0, o1);
           *reinterpret_cast<uint4*>(smem + OFF_KV + d * SUB_KV + sw128_off(key, 2 * part)) = o0;
@@ -339,10 +330,13 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
           *reinterpret_cast<uint4*>(smem + off) = make_uint4(o[0], o[1], o[2], o[3]);
         }
       }
-      if (!PAGED) cp_async_wait_all();
-      fence_async_smem();
-      mbar_arrive(bar(B_QFULL));
-      for (int32_t t = 0; t < it.n_tiles && ok; ++t, ++gtile) ok = gather_tile(it, t, gtile, threadIdx.x);
+      if (!PAGED) {
+        cp_async_arrive_noinc(bar(B_QFULL));
+      } else {
+        fence_async_smem();
+        mbar_arrive(bar(B_QFULL));
+      }
+      for (int32_t t = 0; t < it.n_tiles && ok; ++t, ++gtile) ok = issue(prepare(it, t, threadIdx.x), gtile);
     }
   } else if (warp == MMA_WARP) {
     // ================================================================= MMA issuer
@@ -355,6 +349,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
       for (int32_t item = blockIdx.x, it_n = 0; item < n_items && ok; item += gridDim.x, ++it_n) {
         const Item it = make_item(p, item);
         if (!mbar_wait(bar(B_QFULL), it_n & 1, abort_flag, p.status, p.wait_ns)) break;
+        fence_async_smem();
         tc_fence_after();
         if (it.n_tiles == 0) mma_commit(bar(B_QEMPTY));
         for (int32_t t = 0; t < it.n_tiles && ok; ++t, ++gtile) {
@@ -365,6 +360,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
               ok = false;
               break;
             }
+            fence_async_smem();  // cp.async (generic proxy) writes -> tcgen05.mma (async proxy) reads
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -407,7 +403,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
       const int32_t* idx_row = p.idx + static_cast<int64_t>(it.irow) * p.k;
       if (quad == 0) m_run[hcol + lane] = -INFINITY;
       named_bar(1, SM_THREADS);
-      if (it.n_tiles > 0 && !gather_tile(it, 0, gtile, threadIdx.x)) break;
+      if (it.n_tiles > 0 && !issue(prepare(it, 0, threadIdx.x), gtile)) break;
       float lsum[32];
 #pragma unroll
       for (int h = 0; h < 32; ++h) lsum[h] = 0.f;
@@ -417,6 +413,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         const int32_t v = jj < p.k ? idx_row[jj] : -1;
         const int64_t prow = kv_row<PAGED>(p, it.irow, v, seq_len);
         const bool valid = prow >= 0;
+        Plan next_plan;  // indices of the next tile, loaded while this tile's softmax runs
+        if (t + 1 < it.n_tiles) next_plan = prepare(it, t + 1, threadIdx.x);
         const float kscale = PAGED ? (valid ? p.kv_scale[prow] : 0.f) : 1.f;
         if (!mbar_wait(bar(B_SFULL), par, abort_flag, p.status, p.wait_ns)) {
           ok = false;
@@ -510,7 +508,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(bar(B_PFULL));
-        if (t + 1 < it.n_tiles && !gather_tile(it, t + 1, gtile + 1, threadIdx.x)) {
+        if (t + 1 < it.n_tiles && !issue(next_plan, gtile + 1)) {
           ok = false;
           break;
         }

@@ -27,7 +27,7 @@ from .generators import (
 )
 
 __all__ = ["PrefillSpec", "DecodeSpec", "WORKLOADS", "make_prefill", "make_decode",
-           "decode_context_lengths", "page_table",
+           "decode_context_lengths", "page_table", "make_decode_indexer",
            "IDX_HEADS", "IDX_DIM", "MLA_HEADS", "D_QK", "D_V", "PAGE"]
 
 IDX_HEADS, IDX_DIM = 32, 128
@@ -179,6 +179,17 @@ def _fp8_pool(seed, n_pages, dim, device):
     if device is None:
         return codes.numpy(), sc.numpy()
     return codes, sc
+
+
+def make_decode_indexer(spec: DecodeSpec, layer: int, n_pages: int, batch: int, device=None) -> dict:
+    """Indexer inputs of one Full layer of a decode step: q_idx [B,32,128] bf16, w [B,32] fp32,
+    idx_keys [P,64,128] e4m3 + idx_key_scale [P,64] (streams keyed by the layer number)."""
+    s = spec.seed
+    q = _normal(sub_seed(s, layer, T_QIDX), batch * IDX_HEADS * IDX_DIM, device)
+    w = _f32(_normal(sub_seed(s, layer, T_W), batch * IDX_HEADS, device), device).reshape(batch, IDX_HEADS)
+    keys, sc = _fp8_pool(sub_seed(s, layer, T_KIDX), n_pages, IDX_DIM, device)
+    return {"q_idx": _bf16(q, device).reshape(batch, IDX_HEADS, IDX_DIM), "w": w, "idx_keys": keys,
+            "idx_key_scale": sc}
 
 
 def make_decode(spec: DecodeSpec, device=None, ctx=None, layers=None) -> dict:
