@@ -5,6 +5,8 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
+#include <vector>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -375,12 +377,15 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
 
 // ---------------------------------------------------------------------------- group plan
 
+struct Chunk {
+  int32_t row0, rows;  // query rows [row0, row0 + rows) of the group
+  int64_t ld, max_len; // score row stride and longest candidate row of the chunk
+};
+
 struct GroupPlan {
   bool quant_q = false, quant_k = false;
   size_t off_q8 = 0, off_sq = 0, off_k8 = 0, off_sk = 0, off_scores = 0, off_topk = 0, off_mla = 0, total = 0;
-  int32_t chunk_rows = 0;
-  int64_t ld = 0;
-  int64_t max_len = 0;
+  std::vector<Chunk> chunks;
   size_t topk_ws = 0;
 };
 
@@ -406,19 +411,35 @@ dsa_status plan_group(const dsa_group_args* a, int sms, GroupPlan* g) {
     g->off_k8 = take(static_cast<size_t>(kv.n_tokens) * 128);
     g->off_sk = take(static_cast<size_t>(kv.n_tokens) * 4);
   }
+  // Query-row chunks whose [rows, ld] score block fits the budget: causal rows grow with the
+  // position, so early chunks take more (shorter) rows than late ones.
+  g->chunks.clear();
+  size_t score_floats = 0;
   if (paged) {
-    g->max_len = static_cast<int64_t>(kv.max_pages) * DSA_PAGE;
-    g->ld = g->max_len;
-    g->chunk_rows = static_cast<int32_t>(n);
+    const int64_t len = static_cast<int64_t>(kv.max_pages) * DSA_PAGE;
+    g->chunks.push_back({0, static_cast<int32_t>(n), len, len});
+    score_floats = static_cast<size_t>(n) * len;
   } else {
-    g->max_len = std::min<int64_t>(static_cast<int64_t>(a->q_pos0) + n, kv.n_tokens);
-    g->ld = static_cast<int64_t>(align_up(static_cast<size_t>(std::max<int64_t>(g->max_len, 4)), 4));
-    int64_t c = std::max<int64_t>(16, kScoreBudgetFloats / g->ld);
-    c = c / 16 * 16;
-    g->chunk_rows = static_cast<int32_t>(std::min<int64_t>(c, n));
+    for (int64_t c0 = 0; c0 < n;) {
+      const double a0 = static_cast<double>(a->q_pos0) + static_cast<double>(c0);
+      int64_t c = static_cast<int64_t>((-a0 + std::sqrt(a0 * a0 + 4.0 * kScoreBudgetFloats)) / 2.0);
+      c = std::max<int64_t>(16, c / 16 * 16);
+      c = std::min<int64_t>(c, n - c0);
+      int64_t len = 0, ld = 0;
+      for (;; c -= 16) {
+        len = std::min<int64_t>(static_cast<int64_t>(a->q_pos0) + c0 + c, kv.n_tokens);
+        ld = static_cast<int64_t>(align_up(static_cast<size_t>(std::max<int64_t>(len, 4)), 4));
+        if (c <= 16 || c * ld <= kScoreBudgetFloats) break;
+      }
+      g->chunks.push_back({static_cast<int32_t>(c0), static_cast<int32_t>(c), ld, len});
+      score_floats = std::max(score_floats, static_cast<size_t>(c) * ld);
+      c0 += c;
+    }
   }
-  g->off_scores = take(static_cast<size_t>(g->chunk_rows) * g->ld * 4);
-  g->topk_ws = plan_topk(g->chunk_rows, g->max_len, a->k, sms).ws;
+  g->topk_ws = 0;
+  for (const Chunk& ch : g->chunks)
+    g->topk_ws = std::max(g->topk_ws, plan_topk(ch.rows, ch.max_len, a->k, sms).ws);
+  g->off_scores = take(score_floats * 4);
   g->off_topk = take(g->topk_ws);
   size_t mla_ws = 0;
   const int32_t nq = a->n_idx_rows * a->q_rows_per_idx_row;
@@ -677,14 +698,14 @@ dsa_status indexshare_group_forward(const dsa_group_args* a, dsa_index_handle* h
     float* scores = reinterpret_cast<float*>(ws + g.off_scores);
     const bool paged = keys.block_table != nullptr;
     const size_t qrow_bytes = qdt == DSA_E4M3 ? 32 * 128 : 32 * 128 * 2;
-    for (int32_t c0 = 0; c0 < n; c0 += g.chunk_rows) {
-      const int32_t cn = std::min(g.chunk_rows, n - c0);
+    for (const Chunk& ch : g.chunks) {
+      const int32_t c0 = ch.row0, cn = ch.rows;
       const uint8_t* qc = static_cast<const uint8_t*>(qi) + static_cast<size_t>(c0) * qrow_bytes;
       const float* qsc = qs ? qs + static_cast<size_t>(c0) * 32 : nullptr;
       DSA_TRY(launch_indexer(qc, qdt, qsc, a->w + static_cast<size_t>(c0) * 32, cn, a->q_pos0 + c0, &keys, scores,
-                             g.ld, st));
-      DSA_TRY(launch_topk(scores, g.ld, cn, paged ? keys.seq_lens : nullptr,
-                          static_cast<int64_t>(a->q_pos0) + c0 + 1, g.max_len, a->k,
+                             ch.ld, st));
+      DSA_TRY(launch_topk(scores, ch.ld, cn, paged ? keys.seq_lens : nullptr,
+                          static_cast<int64_t>(a->q_pos0) + c0 + 1, ch.max_len, a->k,
                           h->idx + static_cast<size_t>(c0) * a->k, ws + g.off_topk, g.topk_ws, st));
     }
     h->generation += 1;

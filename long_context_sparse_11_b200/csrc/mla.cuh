@@ -60,7 +60,13 @@ constexpr int MISC_BYTES = M_RED + 1024;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
 constexpr int SM_WARPS = 8, GA_WARPS = 7;  // 16 warps: 4 per SM sub-partition, 128 registers each
 constexpr int SM_THREADS = SM_WARPS * 32, GA_THREADS = GA_WARPS * 32;
-constexpr int NG = SM_THREADS + GA_THREADS;  // threads that gather KV rows (softmax warps help)
+// Threads that gather KV rows.  bf16 cache: the gather warps alone (cp.async issue is the
+// limit, and the softmax warps would join only after their softmax, late for the first
+// sub-tiles).  FP8 cache: the softmax warps help with the load + convert + store.
+template <bool PAGED>
+__host__ __device__ constexpr bool sm_gather() { return PAGED; }
+template <bool PAGED>
+__host__ __device__ constexpr int n_gather() { return sm_gather<PAGED>() ? SM_THREADS + GA_THREADS : GA_THREADS; }
 constexpr int MMA_WARP = SM_WARPS + GA_WARPS;
 constexpr int THREADS = (MMA_WARP + 1) * 32;
 constexpr int TMEM_COLS = 512;
@@ -203,6 +209,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
   float* red = reinterpret_cast<float*>(misc + M_RED);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t n_items = p.n_q * p.n_split;
+  constexpr bool SM_GATHER = sm_gather<PAGED>();
+  constexpr int NG = n_gather<PAGED>();
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), GA_THREADS);
@@ -278,6 +286,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
     } else {
       // each part: 16 e4m3 values of every sub-tile, all 9 loaded before the first wait (loads do
       // not touch shared memory), converted to f16 and stored once the sub-tile pair is free
+#pragma unroll
       for (int i = 0; i < MAXC; ++i) {
         if (pl.dst[i] == 0xFFFFFFFFu) continue;
         const int key = pl.dst[i] >> 2, part = pl.dst[i] & 3;
@@ -286,11 +295,13 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         for (int d = 0; d < NSUB; ++d)
           raw[d] = pl.nb[i] ? __ldg(reinterpret_cast<const uint4*>(pl.src[i] + d * 64)) : make_uint4(0, 0, 0, 0);
         const bool last = i + 1 == MAXC || pl.dst[i + 1 < MAXC ? i + 1 : i] == 0xFFFFFFFFu;
+        // no early return inside the unrolled loop, so raw[] stays in registers
+        bool free_ok = true;
 #pragma unroll
         for (int d = 0; d < NSUB; ++d) {
-          if ((d & 1) == 0 &&
-              !mbar_wait(bar(d < 8 ? B_EMPTY + d / 2 : B_PVDONE), par, abort_flag, p.status, p.wait_ns))
-            return false;
+          if ((d & 1) == 0 && free_ok)
+            free_ok = mbar_wait(bar(d < 8 ? B_EMPTY + d / 2 : B_PVDONE), par, abort_flag, p.status, p.wait_ns);
+          if (!free_ok) continue;
           uint4 o0, o1;
           e4m3x16_to_f16(raw[d], o0, o1);
           *reinterpret_cast<uint4*>(smem + OFF_KV + d * SUB_KV + sw128_off(key, 2 * part)) = o0;
@@ -300,6 +311,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
             mbar_arrive(bar(B_FULL + d));
           }
         }
+        if (!free_ok) return false;
       }
     }
     return true;
@@ -315,19 +327,37 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
       // ---- query row -> 9 K-major sub-tiles (bf16 copy, or bf16 -> f16 for the FP8 cache path)
       if (!mbar_wait(bar(B_QEMPTY), (it_n & 1) ^ 1, abort_flag, p.status, p.wait_ns)) break;
       const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q + static_cast<int64_t>(it.row) * 64 * 576);
-      for (int c = gq; c < 64 * 72; c += GA_THREADS) {
-        const int h = c / 72, ch = c % 72;
-        const uint32_t off = OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7);
-        if (!PAGED) {
-          cp_async16(base + off, qsrc + h * 1152 + ch * 16, 16);
-        } else {
-          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qsrc + h * 1152 + ch * 16));
-          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-          uint32_t o[4];
+      constexpr int QCH = 64 * 72;  // 16-byte chunks of one query row
+      if (!PAGED) {
+        for (int c = gq; c < QCH; c += GA_THREADS) {
+          const int h = c / 72, ch = c % 72;
+          cp_async16(base + OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7), qsrc + h * 1152 + ch * 16, 16);
+        }
+      } else {
+        // batches of QB loads in flight before the first conversion
+        constexpr int QPER = (QCH + GA_THREADS - 1) / GA_THREADS, QB = 3;
+        static_assert(QPER % QB == 0, "query batches");
+        for (int b0 = 0; b0 < QPER; b0 += QB) {
+          uint4 raw[QB];
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            o[i] = pack_pair(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u), true);
-          *reinterpret_cast<uint4*>(smem + off) = make_uint4(o[0], o[1], o[2], o[3]);
+          for (int j = 0; j < QB; ++j) {
+            const int c = gq + (b0 + j) * GA_THREADS;
+            raw[j] = c < QCH ? __ldg(reinterpret_cast<const uint4*>(qsrc + (c / 72) * 1152 + (c % 72) * 16))
+                             : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int j = 0; j < QB; ++j) {
+            const int c = gq + (b0 + j) * GA_THREADS;
+            if (c >= QCH) continue;
+            const int h = c / 72, ch = c % 72;
+            const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              o[i] = pack_pair(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u), true);
+            *reinterpret_cast<uint4*>(smem + OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7)) =
+                make_uint4(o[0], o[1], o[2], o[3]);
+          }
         }
       }
       if (!PAGED) {
@@ -336,7 +366,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         fence_async_smem();
         mbar_arrive(bar(B_QFULL));
       }
-      for (int32_t t = 0; t < it.n_tiles && ok; ++t, ++gtile) ok = issue(prepare(it, t, threadIdx.x), gtile);
+      const int g = SM_GATHER ? threadIdx.x : gq;
+      for (int32_t t = 0; t < it.n_tiles && ok; ++t, ++gtile) ok = issue(prepare(it, t, g), gtile);
     }
   } else if (warp == MMA_WARP) {
     // ================================================================= MMA issuer
@@ -403,7 +434,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
       const int32_t* idx_row = p.idx + static_cast<int64_t>(it.irow) * p.k;
       if (quad == 0) m_run[hcol + lane] = -INFINITY;
       named_bar(1, SM_THREADS);
-      if (it.n_tiles > 0 && !issue(prepare(it, 0, threadIdx.x), gtile)) break;
+      if (SM_GATHER && it.n_tiles > 0 && !issue(prepare(it, 0, threadIdx.x), gtile)) break;
       float lsum[32];
 #pragma unroll
       for (int h = 0; h < 32; ++h) lsum[h] = 0.f;
@@ -414,7 +445,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         const int64_t prow = kv_row<PAGED>(p, it.irow, v, seq_len);
         const bool valid = prow >= 0;
         Plan next_plan;  // indices of the next tile, loaded while this tile's softmax runs
-        if (t + 1 < it.n_tiles) next_plan = prepare(it, t + 1, threadIdx.x);
+        if (SM_GATHER && t + 1 < it.n_tiles) next_plan = prepare(it, t + 1, threadIdx.x);
         const float kscale = PAGED ? (valid ? p.kv_scale[prow] : 0.f) : 1.f;
         if (!mbar_wait(bar(B_SFULL), par, abort_flag, p.status, p.wait_ns)) {
           ok = false;
@@ -508,7 +539,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(bar(B_PFULL));
-        if (t + 1 < it.n_tiles && !issue(next_plan, gtile + 1)) {
+        if (SM_GATHER && t + 1 < it.n_tiles && !issue(next_plan, gtile + 1)) {
           ok = false;
           break;
         }
