@@ -30,6 +30,12 @@ sys.path.insert(0, ROOT)
 METRIC = "query tokens/s per IndexShare group"
 UNIT = "query tokens/s"
 
+# sparse_mla_kernel<bf16>, L=8,192 prefill launch (8,192 query rows): ncu measured 680.9 MB read
+# + 508.7 MB written = 145,213 B per query row (queries 73,728 B in, outputs 65,536 B out, the
+# rest index rows and the latent rows' first touch).
+MLA_DRAM_BYTES_PER_ROW_BF16 = (680.907520e6 + 508.744448e6) / 8192
+
+
 
 def parse():
     p = argparse.ArgumentParser()
@@ -384,10 +390,19 @@ def run_ours(args, ws, rank, local):
     mla_avg = statistics.mean(mla_ms)
     idx_avg = statistics.mean(idx_ms)
     mla_tf = counts["mla_flops_per_layer"] / (mla_avg / 1e3) / 1e12
+    traffic = None
+    if not args.workload.startswith("decode"):
+        # DRAM bytes (read + write) of one bf16 launch grow with the query rows (queries in,
+        # outputs out; the latent rows stay in L2): measured by ncu at 8,192 rows, scaled.
+        traffic = {"bytes_per_launch": round(MLA_DRAM_BYTES_PER_ROW_BF16 * counts["mla_rows"]),
+                   "source": "ncu dram__bytes_read.sum + dram__bytes_write.sum at L=8192, scaled by query rows"}
     mla_roof = {"kernel": "sparse_mla_kernel (a6)", "bound": "tensor", "achieved": round(mla_tf, 1),
                 "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(mla_tf / bf16_peak, 4),
-                "peak_source": f"{peak_kind} bf16 dense (burst)", "traffic": None,
+                "peak_source": f"{peak_kind} bf16 dense (burst)",
+                "traffic": traffic["bytes_per_launch"] if traffic else None,
                 "algorithmic_flops_per_launch": counts["mla_flops_per_layer"], "avg_launch_ms": round(mla_avg, 4)}
+    if traffic:
+        mla_roof["traffic_source"] = traffic["source"]
     phases = {"indexer_topk_ms": round(idx_avg, 4), "mla_ms_per_layer": round(mla_avg, 4),
               "indexer_topk_tflops": round(counts["indexer_flops"] / (idx_avg / 1e3) / 1e12, 1),
               "groups_per_step": n_groups}
