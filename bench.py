@@ -183,6 +183,43 @@ class Workload:
             g.forward()
 
 
+def indexer_alone(wl, spec, dev, stream):
+    """Prefill a2+a3 kernel alone, for its tensor-pipe fraction: the group's indexer query rows in
+    blocks of up to 8,192 rows against all keys (causal), scores into one [rows, L] fp32 block,
+    CUDA events around the launches (outside the timed steps).  FP8 inputs are quantised first,
+    untimed, as the group does on its own."""
+    import torch
+    import long_context_sparse_11_b200 as dsa
+    inp, L = wl.inp, spec.L
+    q, w = inp["q_idx"], inp["w"]
+    q_scale = None
+    if spec.indexer_fp8:
+        q, q_scale = dsa.quant_e4m3(inp["q_idx"])
+        k8, k_scale = dsa.quant_e4m3(inp["k_idx"])
+        keys = dsa.dense_view(k8, k_scale)
+    else:
+        keys = dsa.dense_view(inp["k_idx"])
+    R = min(L, 8192)
+    scores = torch.empty(R, L, dtype=torch.float32, device=dev)
+
+    def run():
+        for r0 in range(0, L, R):
+            n = min(R, L - r0)
+            dsa.indexer_score(q[r0:r0 + n], w[r0:r0 + n], keys, scores[:n],
+                              q_scale=None if q_scale is None else q_scale[r0 * 32:(r0 + n) * 32], q_pos0=r0)
+
+    run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run()
+    e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    del scores
+    return ms, (L + R - 1) // R
+
+
 # ----------------------------------------------------------------------------- clocks
 
 
@@ -421,6 +458,23 @@ def run_ours(args, ws, rank, local):
             phases["mla_roofline"] = mla_roof
     if n_groups > 1:
         phases["step_ms_all_layers"] = round(ms_per_step, 4)
+    if not args.workload.startswith("decode"):
+        # the indexer kernel alone against the tensor peak of its input type (e4m3: the measured
+        # bf16 peak x 2, the nominal fp8 / bf16 ratio), and the IndexShare group against four
+        # independent full layers (each with its own a1-a4), from the same phase timings
+        ia_ms, ia_launches = indexer_alone(wl, wl.spec, dev, stream)
+        ia_tf = counts["indexer_flops"] / (ia_ms / 1e3) / 1e12
+        ia_peak = bf16_peak * (2.0 if wl.spec.indexer_fp8 else 1.0)
+        phases["indexer_alone"] = {"ms": round(ia_ms, 4), "launches": ia_launches, "tflops": round(ia_tf, 1),
+                                   "peak": round(ia_peak, 1), "frac": round(ia_tf / ia_peak, 4),
+                                   "peak_source": f"{peak_kind} bf16 dense (burst)" +
+                                   (" x 2 (fp8 / bf16 nominal)" if wl.spec.indexer_fp8 else "")}
+        nl = wl.layers_per_group[0]
+        group_ms = idx_avg + nl * mla_avg
+        full_ms = nl * (idx_avg + mla_avg)
+        phases["indexshare_vs_independent_full_layers"] = {
+            "group_ms": round(group_ms, 3), "independent_full_layers_ms": round(full_ms, 3),
+            "ratio": round(group_ms / full_ms, 4)}
 
     e2e = None
     if not args.no_e2e:

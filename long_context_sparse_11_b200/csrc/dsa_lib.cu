@@ -389,7 +389,14 @@ struct GroupPlan {
   size_t topk_ws = 0;
 };
 
-constexpr int64_t kScoreBudgetFloats = 16LL << 20;  // 64 MB of scores per chunk (L2-sized)
+// Score block per query chunk: at least 64 MB (L2-sized), and large enough that the last
+// chunks of a long prefill still hold kScoreMinRows rows (fewer, fuller launches), at most 1 GB.
+constexpr int64_t kScoreBudgetFloats = 16LL << 20;
+constexpr int64_t kScoreBudgetMaxFloats = 256LL << 20;
+#ifndef DSA_SCORE_MIN_ROWS
+#define DSA_SCORE_MIN_ROWS 2048
+#endif
+constexpr int64_t kScoreMinRows = DSA_SCORE_MIN_ROWS;
 
 dsa_status plan_group(const dsa_group_args* a, int sms, GroupPlan* g) {
   const dsa_cache_view& kv = a->idx_keys;
@@ -420,16 +427,18 @@ dsa_status plan_group(const dsa_group_args* a, int sms, GroupPlan* g) {
     g->chunks.push_back({0, static_cast<int32_t>(n), len, len});
     score_floats = static_cast<size_t>(n) * len;
   } else {
+    const int64_t longest = std::min<int64_t>(static_cast<int64_t>(a->q_pos0) + n, kv.n_tokens);
+    const int64_t budget = std::min(kScoreBudgetMaxFloats, std::max(kScoreBudgetFloats, kScoreMinRows * longest));
     for (int64_t c0 = 0; c0 < n;) {
       const double a0 = static_cast<double>(a->q_pos0) + static_cast<double>(c0);
-      int64_t c = static_cast<int64_t>((-a0 + std::sqrt(a0 * a0 + 4.0 * kScoreBudgetFloats)) / 2.0);
+      int64_t c = static_cast<int64_t>((-a0 + std::sqrt(a0 * a0 + 4.0 * static_cast<double>(budget))) / 2.0);
       c = std::max<int64_t>(16, c / 16 * 16);
       c = std::min<int64_t>(c, n - c0);
       int64_t len = 0, ld = 0;
       for (;; c -= 16) {
         len = std::min<int64_t>(static_cast<int64_t>(a->q_pos0) + c0 + c, kv.n_tokens);
         ld = static_cast<int64_t>(align_up(static_cast<size_t>(std::max<int64_t>(len, 4)), 4));
-        if (c <= 16 || c * ld <= kScoreBudgetFloats) break;
+        if (c <= 16 || c * ld <= budget) break;
       }
       g->chunks.push_back({static_cast<int32_t>(c0), static_cast<int32_t>(c), ld, len});
       score_floats = std::max(score_floats, static_cast<size_t>(c) * ld);
