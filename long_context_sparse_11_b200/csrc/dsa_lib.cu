@@ -211,6 +211,7 @@ dsa_status launch_indexer(const void* q, int32_t q_dtype, const float* q_scale, 
   p.n_pages = static_cast<int32_t>(keys->n_tokens / DSA_PAGE);
   p.status = ds->status;
   p.wait_ns = static_cast<uint64_t>(g_wait_ns);
+  p.unit_tiles = idx::UNIT_TILES;
   CUtensorMap mq, mk;
   const uint64_t qrows = static_cast<uint64_t>(n_q) * 32;
   if (paged) {
@@ -218,7 +219,11 @@ dsa_status launch_indexer(const void* q, int32_t q_dtype, const float* q_scale, 
     DSA_TRY(make_map(&mk, keys->data, false, 128, static_cast<uint64_t>(keys->n_tokens), 128, 128, 64));
     const int64_t max_len = static_cast<int64_t>(keys->max_pages) * DSA_PAGE;
     const int64_t tiles = (max_len + idx::BLOCK_KEYS - 1) / idx::BLOCK_KEYS;
-    dim3 grid(static_cast<unsigned>((tiles + idx::UNIT_TILES - 1) / idx::UNIT_TILES), static_cast<unsigned>(n_q));
+    // few long sequences: shorter units, so that the grid still covers the SMs several times over
+    int32_t unit = idx::UNIT_TILES;
+    while (unit > 4 && static_cast<int64_t>(n_q) * ((tiles + unit - 1) / unit) < 4LL * ds->sms) unit /= 2;
+    p.unit_tiles = unit;
+    dim3 grid(static_cast<unsigned>((tiles + unit - 1) / unit), static_cast<unsigned>(n_q));
     using C = idx::Cfg<true, true>;
     idx::indexer_kernel<true, true><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, p);
     count_launch();

@@ -21,7 +21,7 @@ namespace dsa {
 namespace idx {
 
 constexpr int BLOCK_KEYS = 128;
-constexpr int UNIT_TILES = 32;  // key tiles per work unit
+constexpr int UNIT_TILES = 32;  // key tiles per work unit (default; decode may use fewer)
 
 template <bool FP8, bool PAGED>
 struct Cfg {
@@ -64,6 +64,7 @@ struct Params {
   int32_t q_pos0;
   int32_t max_pages;
   int32_t n_pages;
+  int32_t unit_tiles;       // key tiles per CTA
   int* status;
   uint64_t wait_ns;
 };
@@ -101,8 +102,8 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
     len = static_cast<int32_t>(l);
   }
   const int32_t n_tiles = (len + BLOCK_KEYS - 1) / BLOCK_KEYS;
-  const int32_t kt0 = blockIdx.x * UNIT_TILES;
-  const int32_t kt1 = min(kt0 + UNIT_TILES, n_tiles);
+  const int32_t kt0 = blockIdx.x * p.unit_tiles;
+  const int32_t kt1 = min(kt0 + p.unit_tiles, n_tiles);
   if (kt0 >= kt1) return;  // uniform across the CTA
 
   // group g needs tile kt iff some of its rows has a candidate in the tile

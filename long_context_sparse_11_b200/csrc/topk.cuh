@@ -267,9 +267,17 @@ __global__ void __launch_bounds__(SEG_THREADS) topk_seg_filter_kernel(const floa
                                                                       int64_t causal_len0, int64_t cap, int32_t k,
                                                                       int32_t seg_len, SegWs ws,
                                                                       int32_t* __restrict__ idx_out) {
+  // The segment's selections and threshold-bin candidates are gathered in shared memory and
+  // placed in the row's arrays with one global reservation each per CTA: a per-element atomic
+  // on the row's counter serialises about k same-address atomics per row.
+  constexpr int SEL_BUF = 2048, CAND_BUF = 1024;
   __shared__ uint32_t hist[BINS];
   __shared__ uint32_t warp_sum[32];
   __shared__ uint32_t sel[3];
+  __shared__ int32_t s_sel[SEL_BUF];
+  __shared__ uint32_t s_ckey[CAND_BUF];
+  __shared__ int32_t s_cidx[CAND_BUF];
+  __shared__ int32_t s_cnt[2], s_base[2];
   const int32_t r = blockIdx.y;
   const int32_t n = row_length(r, row_len, causal_len0, cap);
   if (n <= k) return;
@@ -279,6 +287,7 @@ __global__ void __launch_bounds__(SEG_THREADS) topk_seg_filter_kernel(const floa
   const int t = threadIdx.x;
   const uint32_t* g = ws.hist + static_cast<int64_t>(r) * BINS;
   for (int b = t; b < BINS; b += SEG_THREADS) hist[b] = g[b];
+  if (t == 0) s_cnt[0] = s_cnt[1] = 0;
   __syncthreads();
   find_threshold<SEG_THREADS>(hist, static_cast<uint32_t>(k), warp_sum, &sel[0], &sel[1], &sel[2]);
   const uint32_t T = sel[0], above = sel[1], eq = sel[2];
@@ -293,14 +302,43 @@ __global__ void __launch_bounds__(SEG_THREADS) topk_seg_filter_kernel(const floa
     const uint32_t key = f32_key(row[i]);
     const uint32_t d = key >> 20;
     if (d > T || (take_eq && d == T)) {
-      const int32_t pos = atomicAdd(&cnt[0], 1);
-      if (pos < k) out[pos] = i;
-    } else if (collect && d == T) {
-      const int32_t c = atomicAdd(&cnt[1], 1);
-      if (c < ws.gcap) {
-        ck[c] = key;
-        ci[c] = i;
+      const int32_t p = atomicAdd(&s_cnt[0], 1);
+      if (p < SEL_BUF) {
+        s_sel[p] = i;
+      } else {  // overflow (a segment holding more than SEL_BUF selections): place directly
+        const int32_t pos = atomicAdd(&cnt[0], 1);
+        if (pos < k) out[pos] = i;
       }
+    } else if (collect && d == T) {
+      const int32_t p = atomicAdd(&s_cnt[1], 1);
+      if (p < CAND_BUF) {
+        s_ckey[p] = key;
+        s_cidx[p] = i;
+      } else {
+        const int32_t c = atomicAdd(&cnt[1], 1);
+        if (c < ws.gcap) {
+          ck[c] = key;
+          ci[c] = i;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const int32_t n_sel = min(s_cnt[0], SEL_BUF), n_cand = min(s_cnt[1], CAND_BUF);
+  if (t == 0) {
+    s_base[0] = n_sel > 0 ? atomicAdd(&cnt[0], n_sel) : 0;
+    s_base[1] = n_cand > 0 ? atomicAdd(&cnt[1], n_cand) : 0;
+  }
+  __syncthreads();
+  for (int32_t j = t; j < n_sel; j += SEG_THREADS) {
+    const int32_t pos = s_base[0] + j;
+    if (pos < k) out[pos] = s_sel[j];
+  }
+  for (int32_t j = t; j < n_cand; j += SEG_THREADS) {
+    const int32_t c = s_base[1] + j;
+    if (c < ws.gcap) {
+      ck[c] = s_ckey[j];
+      ci[c] = s_cidx[j];
     }
   }
 }
