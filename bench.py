@@ -43,7 +43,8 @@ def parse():
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--workload", default="prefill_32k",
-                   choices=["tiny_prefill", "prefill_32k", "prefill_128k_fp8", "decode_b32_mtp4", "decode_1m_mtp5"])
+                   choices=["tiny_prefill", "prefill_32k", "prefill_128k_fp8", "decode_b32_mtp4", "decode_b32_d0",
+                            "decode_1m_mtp5"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     p.add_argument("--ref-seconds", type=float, default=150.0, help="reference arm total budget")
@@ -450,6 +451,14 @@ def run_ours(args, ws, rank, local):
         phases["indexer_topk_hbm_frac"] = round(gbs / hbm, 4)
         mla_gbs = counts["mla_bytes_per_layer"] / (mla_avg / 1e3) / 1e9
         phases["mla_gbs"] = round(mla_gbs, 1)
+        if wl.spec.rows_per_seq == 1:
+            # one row per sequence: 139,264 flops per 580 gathered bytes, a memory-bound kernel
+            mla_roof = {"kernel": "sparse_mla_kernel<paged e4m3> (a6, a7)", "bound": "hbm",
+                        "achieved": round(mla_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(mla_gbs / hbm, 4),
+                        "peak_source": f"{peak_kind} HBM copy", "traffic": None,
+                        "algorithmic_bytes_per_launch": counts["mla_bytes_per_layer"],
+                        "avg_launch_ms": round(mla_avg, 4)}
+            roofline = mla_roof
         if idx_avg * n_groups > mla_avg * sum(wl.layers_per_group):
             roofline = {"kernel": "indexer_kernel<e4m3,paged> + topk (a2-a4)", "bound": "hbm",
                         "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),

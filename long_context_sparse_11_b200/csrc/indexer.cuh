@@ -33,7 +33,7 @@ struct Cfg {
   static constexpr int KH = FP8 ? 1 : 2;          // 128-byte K halves per row
   static constexpr int KSTEPS = FP8 ? 4 : 8;
   static constexpr int STAGES = FP8 ? 4 : 2;
-  static constexpr int EPI_WARPS = PAGED ? 4 : 8;
+  static constexpr int EPI_WARPS = PAGED ? 4 : 16;
   static constexpr int THREADS = 64 + EPI_WARPS * 32;
   static constexpr int Q_HALF_BYTES = N * 128;    // one K half of one query group
   static constexpr int Q_BYTES = NGROUP * KH * Q_HALF_BYTES;
@@ -237,8 +237,8 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
     // ---------------------------------------------------------------- epilogue warps
     const int e = warp - 2;
     const int quad = warp & 3;
-    const int half = e / 4;                      // prefill: which 4 queries of the group
-    constexpr int QPW = PAGED ? 1 : C::NQ / 2;   // queries per warp per accumulator
+    const int part = e / 4;                      // prefill: which queries of the group
+    constexpr int QPW = PAGED ? 1 : C::NQ / (C::EPI_WARPS / 4);  // queries per warp per accumulator
     const int key_in_tile = quad * 32 + lane;
     int job = 0;
     bool ok = true;
@@ -285,19 +285,28 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
           }
         };
         const uint32_t trow = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + bf * C::N;
-        const int q0 = PAGED ? 0 : half * QPW;
-        // TMEM loads run one query ahead of the math
+        const int q0 = PAGED ? 0 : part * QPW;
         uint32_t xa[32], xb[32];
-        DSA_TMEM_LD_X32_NOWAIT(trow + q0 * 32, xa);
+        if constexpr (QPW == 2) {
+          // both queries' accumulators in flight at once: one TMEM load latency per group
+          DSA_TMEM_LD_X32_NOWAIT(trow + q0 * 32, xa);
+          DSA_TMEM_LD_X32_NOWAIT(trow + (q0 + 1) * 32, xb);
+          DSA_TMEM_WAIT_LD2(xa, xb);
+          score(xa, q0);
+          score(xb, q0 + 1);
+        } else {
+          // TMEM loads run one query ahead of the math
+          DSA_TMEM_LD_X32_NOWAIT(trow + q0 * 32, xa);
 #pragma unroll
-        for (int j = 0; j < QPW; j += 2) {
-          DSA_TMEM_WAIT_LD(xa);
-          if (j + 1 < QPW) DSA_TMEM_LD_X32_NOWAIT(trow + (q0 + j + 1) * 32, xb);
-          score(xa, q0 + j);
-          if (j + 1 < QPW) {
-            DSA_TMEM_WAIT_LD(xb);
-            if (j + 2 < QPW) DSA_TMEM_LD_X32_NOWAIT(trow + (q0 + j + 2) * 32, xa);
-            score(xb, q0 + j + 1);
+          for (int j = 0; j < QPW; j += 2) {
+            DSA_TMEM_WAIT_LD(xa);
+            if (j + 1 < QPW) DSA_TMEM_LD_X32_NOWAIT(trow + (q0 + j + 1) * 32, xb);
+            score(xa, q0 + j);
+            if (j + 1 < QPW) {
+              DSA_TMEM_WAIT_LD(xb);
+              if (j + 2 < QPW) DSA_TMEM_LD_X32_NOWAIT(trow + (q0 + j + 2) * 32, xa);
+              score(xb, q0 + j + 1);
+            }
           }
         }
         tc_fence_before();

@@ -206,6 +206,23 @@ __host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c) {
                :                                                                                              \
                : "memory")
 
+// No instruction: orders a second load's registers after a preceding DSA_TMEM_WAIT_LD (which
+// waits for all of the thread's outstanding TMEM loads), so the compiler reads them no earlier.
+#define DSA_TMEM_TIE(r)                                                                                       \
+  asm volatile(""                                                                                             \
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),         \
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),      \
+                 "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),   \
+                 "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),   \
+                 "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])                                           \
+               :                                                                                              \
+               : "memory")
+#define DSA_TMEM_WAIT_LD2(a, b) \
+  do {                          \
+    DSA_TMEM_WAIT_LD(a);        \
+    DSA_TMEM_TIE(b);            \
+  } while (0)
+
 // (a0, a1) += (w0, w1) * (x0, x1) as one packed fp32 FMA (fma.rn.f32x2).
 __device__ __forceinline__ void ffma2(float& a0, float& a1, float w0, float w1, float x0, float x1) {
   asm("{\n\t.reg .b64 A, W, X;\n\tmov.b64 A, {%0, %1};\n\tmov.b64 W, {%2, %3};\n\tmov.b64 X, {%4, %5};\n\t"

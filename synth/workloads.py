@@ -10,6 +10,9 @@ Workloads, named by what they are:
                       quantised to e4m3 on the path; MLA latent KV bf16.
 * ``decode_b32_mtp4`` 32 sequences, context ~U[65,536, 262,144], 1 + 4 draft rows per
                       sequence, FP8 paged caches (64-token pages, physically permuted).
+* ``decode_b32_d0``   the same batch and caches as ``decode_b32_mtp4`` with one query row per
+                      sequence (no draft rows): sparse MLA reads 580 B per selected key for 139,264
+                      flops, so it is bound by memory rather than by the tensor cores.
 * ``decode_1m_mtp5``  1 sequence of 1,048,576 tokens, 1 + 5 rows, 78-layer schedule.
 
 Stream ids keep every tensor independent: ``sub_seed(seed, layer, TENSOR_ID)``.
@@ -71,6 +74,7 @@ WORKLOADS = {
     "prefill_128k_fp8": PrefillSpec("prefill_128k_fp8", L=131072, k=2048, seed=3, indexer_fp8=True),
     "decode_b32_mtp4": DecodeSpec("decode_b32_mtp4", batch=32, ctx_lo=65536, ctx_hi=262144,
                                   rows_per_seq=5, seed=4),
+    "decode_b32_d0": DecodeSpec("decode_b32_d0", batch=32, ctx_lo=65536, ctx_hi=262144, rows_per_seq=1, seed=4),
     "decode_1m_mtp5": DecodeSpec("decode_1m_mtp5", batch=1, ctx_lo=1 << 20, ctx_hi=1 << 20,
                                  rows_per_seq=6, seed=5, n_layers=78, fixed_ctx=1 << 20),
 }
