@@ -123,6 +123,21 @@ def test_topk_exact_on_given_scores(rows, L, k):
         assert (got[r][min(k, n):] == -1).all()
 
 
+def test_topk_segmented_crowded_threshold_bin():
+    """Segmented mode (few long rows) where one segment holds thousands of candidates equal to the
+    k-th score: the per-CTA candidate buffer overflows and the rest take the direct path."""
+    rows, L, k = 2, 100000, 2048
+    s = np.round(normal_np(77, 0, rows * L).reshape(rows, L) * 64) / 64
+    s[0, 20000:24000] = 2.5                 # fewer than k scores lie above 2.5 in a N(0,1) row
+    s[1, 50000:56000] = 2.25
+    s = s.astype(np.float32)
+    out = dsa.topk(f32_dev(s), k, row_len=i32_dev(np.full(rows, L, dtype=np.int32)), max_len=L)
+    got = out.cpu().numpy()
+    for r in range(rows):
+        ref = O.topk_row(s[r].astype(np.float64), L, k)
+        assert set(got[r]) == set(ref), r
+
+
 def test_topk_causal_lengths():
     rows, L, k = 64, 600, 256
     s = normal_np(3, 0, rows * L).reshape(rows, L).astype(np.float32)
@@ -193,6 +208,27 @@ def test_indexer_decode_paged():
         ref = O.indexer_scores(qv[b:b + 1], inp["w"][b:b + 1], keys, [n])[0]
         assert np.max(np.abs(got[b, :n] - ref[:n])) <= 2e-5 * np.max(np.abs(ref[:n])) + 1e-6
         assert np.all(np.isnan(got[b, n:]))
+
+
+def test_indexer_decode_paged_one_long_sequence():
+    """One 200K-token sequence: the launch splits its keys into short units (4 tiles per CTA)."""
+    spec = DecodeSpec("t", batch=1, ctx_lo=1, ctx_hi=1, rows_per_seq=1, k=64, n_layers=1, seed=23)
+    ctx = np.array([200003])
+    inp = make_decode(spec, ctx=ctx)
+    bt = inp["block_table"]
+    q8, sq = O.quantize_e4m3_rows(inp["q_idx"], 128)
+    ld = bt.shape[1] * 64
+    scores = torch.full((1, ld), float("nan"), device=DEV)
+    view = dsa.paged_view(u8_dev(inp["idx_keys"]), f32_dev(inp["idx_key_scale"]), i32_dev(bt), i32_dev(ctx))
+    dsa.indexer_score(u8_dev(q8), f32_dev(inp["w"]), view, scores, q_scale=f32_dev(sq))
+    dsa.sync_status()
+    got = scores.cpu().numpy()[0]
+    n = int(ctx[0])
+    qv = O.e4m3_to_f64(q8) * sq.reshape(1, 32, 1)
+    keys = O.paged_rows(inp["idx_keys"], inp["idx_key_scale"], bt[0], n)
+    ref = O.indexer_scores(qv, inp["w"], keys, [n])[0]
+    assert np.max(np.abs(got[:n] - ref[:n])) <= 2e-5 * np.max(np.abs(ref[:n])) + 1e-6
+    assert np.all(np.isnan(got[n:]))
 
 
 # ----------------------------------------------------------------------------- a6
