@@ -28,9 +28,9 @@
 // kind::f16 on f16 operands, exact for e4m3 values; the per-token scale is applied to the
 // logits and folded into P^T).
 //
-// Warps 0-7: softmax / output (warp w: lane quadrant w%4, heads 32*(w/4) .. +31), and part of
-// the next tile's gather; warps 8-14: query rows and the rest of the gather; warp 15: TMEM
-// owner + MMA issuer.  16 warps = 4 per SM sub-partition, so each thread may use 128 registers.
+// Warps 0..SM_WARPS-1: softmax / output (warp w: lane quadrant w%4, HPW heads from HPW*(w/4)),
+// and on the FP8 path part of the gather; the next 7 warps: query rows and the KV gather; the
+// last warp: TMEM owner + MMA issuer.
 #pragma once
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -58,7 +58,14 @@ constexpr int M_LTOT = M_ALPHA + 256;
 constexpr int M_RED = M_LTOT + 256;  // float[4 quadrants][64 heads]
 constexpr int MISC_BYTES = M_RED + 1024;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
-constexpr int SM_WARPS = 8, GA_WARPS = 7;  // 16 warps: 4 per SM sub-partition, 128 registers each
+#ifndef DSA_MLA_SM_WARPS
+#define DSA_MLA_SM_WARPS 16
+#endif
+// softmax warps: 4 lane quadrants x (64 / HPW) head groups; with 8 (16 warps in all, 4 per SM
+// sub-partition) each thread may use 128 registers, with 16 (24 warps) 80
+constexpr int SM_WARPS = DSA_MLA_SM_WARPS, GA_WARPS = 7;
+constexpr int HPW = 64 / (SM_WARPS / 4);  // heads per softmax warp
+static_assert(HPW == 16 || HPW == 32, "softmax warps: 8 or 16");
 constexpr int SM_THREADS = SM_WARPS * 32, GA_THREADS = GA_WARPS * 32;
 // Threads that gather KV rows.  bf16 cache: the gather warps alone (cp.async issue is the
 // limit, and the softmax warps would join only after their softmax, late for the first
@@ -124,6 +131,57 @@ __device__ __forceinline__ float warp_reduce32(const float (&v)[32], int lane) {
     }
   }
   return a[0];
+}
+
+// Max (or sum) over the 32 lanes of a warp for 16 per-lane values; lanes 2i and 2i+1 end with
+// the result for value index i.
+template <bool MAX>
+__device__ __forceinline__ float warp_reduce16(const float (&v)[16], int lane) {
+  float a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool hi = lane & 16;
+    const float keep = hi ? v[8 + i] : v[i];
+    const float give = hi ? v[i] : v[8 + i];
+    const float o = __shfl_xor_sync(0xffffffffu, give, 16);
+    a[i] = MAX ? fmaxf(keep, o) : keep + o;
+  }
+#pragma unroll
+  for (int w = 8, bit = 8; w >= 2; w >>= 1, bit >>= 1) {
+#pragma unroll
+    for (int i = 0; i < w / 2; ++i) {
+      const bool hi = lane & bit;
+      const float keep = hi ? a[w / 2 + i] : a[i];
+      const float give = hi ? a[i] : a[w / 2 + i];
+      const float o = __shfl_xor_sync(0xffffffffu, give, bit);
+      a[i] = MAX ? fmaxf(keep, o) : keep + o;
+    }
+  }
+  const float o = __shfl_xor_sync(0xffffffffu, a[0], 1);
+  return MAX ? fmaxf(a[0], o) : a[0] + o;
+}
+
+// Per-warp head reduction for HPW values: the result for head index i of the warp's group is
+// held by lane reduce_lane(i) (32 values: lane i; 16 values: lanes 2i, 2i+1).
+template <bool MAX, int N>
+__device__ __forceinline__ float warp_reduce_heads(const float (&v)[N], int lane) {
+  if constexpr (N == 32) return warp_reduce32<MAX>(v, lane);
+  else return warp_reduce16<MAX>(v, lane);
+}
+template <int N>
+__device__ __forceinline__ int reduce_head_of_lane(int lane) { return N == 32 ? lane : lane >> 1; }
+template <int N>
+__device__ __forceinline__ bool reduce_lane_writes(int lane) { return N == 32 || (lane & 1) == 0; }
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_heads(uint32_t taddr, uint32_t (&x)[N]) {
+  if constexpr (N == 32) { DSA_TMEM_LD_X32(taddr, x); }
+  else { DSA_TMEM_LD_X16(taddr, x); }
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_heads(uint32_t taddr, const uint32_t (&x)[N]) {
+  if constexpr (N == 32) { DSA_TMEM_ST_X32(taddr, x); }
+  else { DSA_TMEM_ST_X16(taddr, x); }
 }
 
 // Physical cache row of idx value v of sequence seq, or -1 when v is not a valid token.
@@ -218,7 +276,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
     mbar_init(bar(B_SFULL), 1);
     mbar_init(bar(B_PFULL), SM_THREADS);
     mbar_init(bar(B_PVDONE), 1);
-    for (int d = 0; d < NSUB; ++d) mbar_init(bar(B_FULL + d), NG);
+    // every gathering thread that owns a chunk arrives once per sub-tile (FP8: 512 parts per tile)
+    for (int d = 0; d < NSUB; ++d) mbar_init(bar(B_FULL + d), PAGED ? (NG < 512 ? NG : 512) : NG);
     for (int g = 0; g < 4; ++g) mbar_init(bar(B_EMPTY + g), 1);
     *abort_flag = 0;
     need_flags[0] = 0;
@@ -420,24 +479,25 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
       }
     }
   } else {
-    // ================================================================= softmax / output warps 0-7
+    // ================================================================= softmax / output warps
     const int quad = warp & 3, hh = warp >> 2;
     const int key = quad * 32 + lane;                 // TMEM lane: key of S^T, dim of an O^T block
-    const int st = warp * 32 + lane;                  // 0..255
+    const int st = warp * 32 + lane;                  // 0..SM_THREADS-1
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t hcol = 32u * hh;
+    const uint32_t hcol = static_cast<uint32_t>(HPW) * hh;
+    const bool head_lane = lane < HPW;                // lanes that own one of the warp's heads
     uint32_t gtile = 0;
     bool ok = true;
     for (int32_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       const Item it = make_item(p, item);
       const int32_t seq_len = PAGED ? p.seq_lens[it.irow] : 0;
       const int32_t* idx_row = p.idx + static_cast<int64_t>(it.irow) * p.k;
-      if (quad == 0) m_run[hcol + lane] = -INFINITY;
+      if (quad == 0 && head_lane) m_run[hcol + lane] = -INFINITY;
       named_bar(1, SM_THREADS);
       if (SM_GATHER && it.n_tiles > 0 && !issue(prepare(it, 0, threadIdx.x), gtile)) break;
-      float lsum[32];
+      float lsum[HPW];
 #pragma unroll
-      for (int h = 0; h < 32; ++h) lsum[h] = 0.f;
+      for (int h = 0; h < HPW; ++h) lsum[h] = 0.f;
       for (int32_t t = 0; t < it.n_tiles; ++t, ++gtile) {
         const uint32_t par = gtile & 1;
         const int32_t jj = (it.j0 + t) * TILE + key;
@@ -452,20 +512,20 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
           break;
         }
         tc_fence_after();
-        float z[32];
+        float z[HPW];
         {
-          uint32_t x[32];
-          DSA_TMEM_LD_X32(tmem + TM_S + 64u * par + hcol + lane_off, x);
+          uint32_t x[HPW];
+          tmem_ld_heads<HPW>(tmem + TM_S + 64u * par + hcol + lane_off, x);
           const float zs = p.scale_log2 * kscale;
 #pragma unroll
-          for (int h = 0; h < 32; ++h) z[h] = valid ? __uint_as_float(x[h]) * zs : -INFINITY;
+          for (int h = 0; h < HPW; ++h) z[h] = valid ? __uint_as_float(x[h]) * zs : -INFINITY;
         }
         // Lazy running max: the cross-lane reduction is needed only when some logit exceeds
         // its head's running max by more than 8 (log2 units) -- always on an item's first tile.
         volatile int* need = need_flags + (gtile & 1);
         bool exceed = false;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < HPW / 4; ++c) {
           const float4 m4 = *reinterpret_cast<const float4*>(m_run + hcol + 4 * c);
           exceed |= (z[4 * c] > m4.x + 8.f) | (z[4 * c + 1] > m4.y + 8.f) | (z[4 * c + 2] > m4.z + 8.f) |
                     (z[4 * c + 3] > m4.w + 8.f);
@@ -475,9 +535,10 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         if (st == 0) need_flags[(gtile + 1) & 1] = 0;  // the next tile's flag: its readers are done
         const bool resc = *need != 0;
         if (resc) {
-          red[quad * 64 + hcol + lane] = warp_reduce32<true>(z, lane);
+          const float wmax = warp_reduce_heads<true, HPW>(z, lane);
+          if (reduce_lane_writes<HPW>(lane)) red[quad * 64 + hcol + reduce_head_of_lane<HPW>(lane)] = wmax;
           named_bar(1, SM_THREADS);
-          if (quad == 0) {
+          if (quad == 0 && head_lane) {
             const int h = hcol + lane;
             const float tmax = fmaxf(fmaxf(red[h], red[64 + h]), fmaxf(red[128 + h], red[192 + h]));
             const float mo = m_run[h];
@@ -490,7 +551,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
           }
           named_bar(1, SM_THREADS);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < HPW / 4; ++c) {
             const float4 a4 = *reinterpret_cast<const float4*>(alpha + hcol + 4 * c);
             lsum[4 * c] *= a4.x;
             lsum[4 * c + 1] *= a4.y;
@@ -500,7 +561,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         }
         // probabilities 8 heads at a time -> one 16-byte chunk of this key's P^T row
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < HPW / 8; ++c) {
           float m8[8];
           const float4 ma = *reinterpret_cast<const float4*>(m_run + hcol + 8 * c);
           const float4 mb = *reinterpret_cast<const float4*>(m_run + hcol + 8 * c + 4);
@@ -517,7 +578,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
             lsum[h + 1] += p1;
             pk[e] = pack_pair(p0 * kscale, p1 * kscale, PAGED);
           }
-          *reinterpret_cast<uint4*>(smem + OFF_P + sw128_off(key, 4 * hh + c)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(smem + OFF_P + sw128_off(key, (HPW / 8) * hh + c)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
         if (resc && t > 0) {
           // O^T (dims on lanes, heads on columns) *= alpha; PV of the previous tile is done
@@ -528,12 +590,12 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
           tc_fence_after();
 #pragma unroll 1
           for (int mb = 0; mb < 4; ++mb) {
-            uint32_t x[32];
+            uint32_t x[HPW];
             const uint32_t ta = tmem + 64u * mb + hcol + lane_off;
-            DSA_TMEM_LD_X32(ta, x);
+            tmem_ld_heads<HPW>(ta, x);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) x[c] = __float_as_uint(__uint_as_float(x[c]) * alpha[hcol + c]);
-            DSA_TMEM_ST_X32(ta, x);
+            for (int c = 0; c < HPW; ++c) x[c] = __float_as_uint(__uint_as_float(x[c]) * alpha[hcol + c]);
+            tmem_st_heads<HPW>(ta, x);
           }
         }
         fence_async_smem();
@@ -550,9 +612,12 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         if (!mbar_wait(bar(B_PVDONE), (gtile - 1) & 1, abort_flag, p.status, p.wait_ns)) break;
         tc_fence_after();
       }
-      red[quad * 64 + hcol + lane] = warp_reduce32<false>(lsum, lane);
+      {
+        const float wsum = warp_reduce_heads<false, HPW>(lsum, lane);
+        if (reduce_lane_writes<HPW>(lane)) red[quad * 64 + hcol + reduce_head_of_lane<HPW>(lane)] = wsum;
+      }
       named_bar(1, SM_THREADS);
-      if (quad == 0) {
+      if (quad == 0 && head_lane) {
         const int h = hcol + lane;
         l_tot[h] = red[h] + red[64 + h] + red[128 + h] + red[192 + h];
       }
@@ -561,15 +626,15 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         uint16_t* orow = p.out + static_cast<int64_t>(it.row) * 64 * 512;
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
-          uint32_t x[32];
+          uint32_t x[HPW];
           if (it.n_tiles > 0) {
-            DSA_TMEM_LD_X32(tmem + 64u * mb + hcol + lane_off, x);
+            tmem_ld_heads<HPW>(tmem + 64u * mb + hcol + lane_off, x);
           } else {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) x[c] = 0u;
+            for (int c = 0; c < HPW; ++c) x[c] = 0u;
           }
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
+          for (int c = 0; c < HPW; ++c) {
             const int h = hcol + c;
             const float l = l_tot[h];
             const float o = l > 0.f ? __uint_as_float(x[c]) / l : 0.f;
@@ -577,7 +642,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
             orow[h * 512 + mb * 128 + key] = *reinterpret_cast<const uint16_t*>(&ob);
           }
         }
-        if (p.lse && quad == 0) {
+        if (p.lse && quad == 0 && head_lane) {
           const int h = hcol + lane;
           const float l = l_tot[h];
           p.lse[static_cast<int64_t>(it.row) * 64 + h] =
@@ -588,17 +653,17 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         float* po = p.part_o + pr * 64 * 512;
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
-          uint32_t x[32];
+          uint32_t x[HPW];
           if (it.n_tiles > 0) {
-            DSA_TMEM_LD_X32(tmem + 64u * mb + hcol + lane_off, x);
+            tmem_ld_heads<HPW>(tmem + 64u * mb + hcol + lane_off, x);
           } else {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) x[c] = 0u;
+            for (int c = 0; c < HPW; ++c) x[c] = 0u;
           }
 #pragma unroll
-          for (int c = 0; c < 32; ++c) po[(hcol + c) * 512 + mb * 128 + key] = __uint_as_float(x[c]);
+          for (int c = 0; c < HPW; ++c) po[(hcol + c) * 512 + mb * 128 + key] = __uint_as_float(x[c]);
         }
-        if (quad == 0) {
+        if (quad == 0 && head_lane) {
           const int h = hcol + lane;
           p.part_ml[pr * 128 + h] = m_run[h];
           p.part_ml[pr * 128 + 64 + h] = l_tot[h];

@@ -183,6 +183,23 @@ __host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c) {
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])                      \
       : "memory")
 
+#define DSA_TMEM_LD_X16(taddr, r)                                                                             \
+  asm volatile(                                                                                               \
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t" \
+      "tcgen05.wait::ld.sync.aligned;"                                                                        \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),       \
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])  \
+      : "r"(taddr)                                                                                            \
+      : "memory")
+
+#define DSA_TMEM_ST_X16(taddr, r)                                                                             \
+  asm volatile(                                                                                               \
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t" \
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),                                                          \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),      \
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])                       \
+      : "memory")
+
 // TMEM load without the wait, and a wait that names the destination registers so that no use
 // of them can be scheduled before it (lets one load overlap the math on the previous one).
 #define DSA_TMEM_LD_X32_NOWAIT(taddr, r)                                                                      \
