@@ -63,7 +63,10 @@ constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
 #endif
 // softmax warps: 4 lane quadrants x (64 / HPW) head groups; with 8 (16 warps in all, 4 per SM
 // sub-partition) each thread may use 128 registers, with 16 (24 warps) 80
-constexpr int SM_WARPS = DSA_MLA_SM_WARPS, GA_WARPS = 7;
+#ifndef DSA_MLA_GA_WARPS
+#define DSA_MLA_GA_WARPS 7
+#endif
+constexpr int SM_WARPS = DSA_MLA_SM_WARPS, GA_WARPS = DSA_MLA_GA_WARPS;
 constexpr int HPW = 64 / (SM_WARPS / 4);  // heads per softmax warp
 static_assert(HPW == 16 || HPW == 32, "softmax warps: 8 or 16");
 constexpr int SM_THREADS = SM_WARPS * 32, GA_THREADS = GA_WARPS * 32;
@@ -394,8 +397,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         }
       } else {
         // batches of QB loads in flight before the first conversion
-        constexpr int QPER = (QCH + GA_THREADS - 1) / GA_THREADS, QB = 3;
-        static_assert(QPER % QB == 0, "query batches");
+        constexpr int QPER = (QCH + GA_THREADS - 1) / GA_THREADS, QB = 3;  // chunks c >= QCH are skipped
         for (int b0 = 0; b0 < QPER; b0 += QB) {
           uint4 raw[QB];
 #pragma unroll
