@@ -141,3 +141,41 @@ def test_decode_group_mtp_paged():
                 ref, _ = O.sparse_mla_row(O.bf16_to_f64(inp["Q"][l][row]), kv, idx[b], inp["softmax_scale"])
                 ma, rel = attn_errors(outs[l][row], ref)
                 assert ma <= 2e-2 and rel <= 5e-3, (l, row, ma, rel)
+
+
+def test_decode_group_replays_from_a_captured_cuda_graph():
+    """The group call allocates nothing and uses only the caller's stream: captured once as a CUDA
+    graph and replayed on new query rows, it gives what eager calls give on them (the same Top-k
+    sets; the order inside a row is unspecified, so the attention sums may differ in rounding)."""
+    spec = DecodeSpec("g", batch=4, ctx_lo=300, ctx_hi=9000, rows_per_seq=3, k=256, n_layers=2, seed=9)
+    inp = make_decode(spec)
+    ctx_d, bt_d = i32_dev(inp["ctx"]), i32_dev(inp["block_table"])
+    keys = dsa.paged_view(u8_dev(inp["idx_keys"]), f32_dev(inp["idx_key_scale"]), bt_d, ctx_d)
+    kvs = [dsa.paged_view(u8_dev(inp["KV"][l]), f32_dev(inp["KV_scale"][l]), bt_d, ctx_d) for l in range(2)]
+    q_idx, w, Q = bf16_dev(inp["q_idx"]), f32_dev(inp["w"]), [bf16_dev(x) for x in inp["Q"]]
+    g = dsa.IndexShareGroup(q_idx, w, keys, spec.k, Q, kvs, inp["softmax_scale"], indexer_dtype=dsa.DSA_E4M3,
+                            q_rows_per_idx_row=spec.rows_per_seq)
+    g.forward()                                   # first call (library set-up) outside the capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        g.forward()
+    # new step inputs in place, then replay vs eager on the same inputs
+    gen = torch.Generator(device="cpu").manual_seed(5)
+    q_idx.copy_(torch.randn(q_idx.shape, generator=gen).to(torch.bfloat16))
+    for q in Q:
+        q.copy_(torch.randn(q.shape, generator=gen).to(torch.bfloat16))
+    graph.replay()
+    torch.cuda.synchronize()
+    dsa.sync_status()
+    got_idx = g.idx.clone()
+    got = [o.clone() for o in g.out] + [x.clone() for x in g.lse]
+    g.forward()
+    dsa.sync_status()
+    assert torch.equal(torch.sort(got_idx, dim=1).values, torch.sort(g.idx, dim=1).values)
+    for a, b in zip(got[:2], g.out):
+        ma, rel = attn_errors(a.float().cpu().numpy().astype(np.float64), b.float().cpu().numpy().astype(np.float64))
+        assert ma <= 2e-2 and rel <= 1e-3, (ma, rel)
+    for a, b in zip(got[2:], g.lse):
+        assert torch.max(torch.abs(a - b)).item() <= 1e-3
+    del graph
