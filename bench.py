@@ -521,9 +521,25 @@ def run_ours(args, ws, rank, local):
             "group_ms": round(group_ms, 3), "independent_full_layers_ms": round(full_ms, 3),
             "ratio": round(group_ms / full_ms, 4)}
 
+    def make_twin():
+        """A second set of device inputs/outputs (the same seeded data), so that one step's upload
+        can run while the previous step computes; None when the GPU has no room for it."""
+        free, _ = torch.cuda.mem_get_info()
+        if free < 1.25 * torch.cuda.memory_allocated() + (4 << 30):
+            return None
+        wl2 = Workload(spec, args.workload, dev)
+        wl2.forward()
+        g2 = None
+        if graph is not None:
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2):
+                wl2.forward()
+        torch.cuda.synchronize()
+        return wl2, (g2.replay if g2 is not None else wl2.forward), g2
+
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, wl, stream, ws, run_step)
+        e2e = run_e2e(args, wl, stream, ws, run_step, make_twin)
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline and ws == 1:
@@ -543,45 +559,53 @@ def run_ours(args, ws, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, wl, stream, ws, run_step):
+def run_e2e(args, wl, stream, ws, run_step, make_twin=None):
     """Same metric through the public API with host buffers: every step copies its inputs from
-    pinned host memory to the device, runs the groups and reads the outputs back.  The copies run
-    on their own streams, so a step's input upload overlaps the previous step's result download
-    (the two PCIe directions); each step's compute waits for its inputs and for the previous
-    download to have drained the output buffers."""
+    pinned host memory to the device, runs the groups and reads the outputs back.  Uploads and
+    downloads run on their own streams; with a second set of device buffers (when the GPU has room)
+    consecutive steps alternate between the two sets, so step i+1's upload overlaps step i's
+    compute and step i-1's download.  A step's compute waits for its own upload and for the download
+    of the outputs its buffer set held two steps earlier."""
     import torch
     import long_context_sparse_11_b200 as dsa
-    dev_in = wl.step_inputs
-    host_in = [t.cpu().pin_memory() for t in dev_in]
-    outs = wl.outputs
-    host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
+    host_in = [t.cpu().pin_memory() for t in wl.step_inputs]
+    host_out = [torch.empty_like(o, device="cpu").pin_memory() for o in wl.outputs]
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
     steps = max(2, min(args.steps, 5))
+    sets = [(wl, run_step)]
+    twin = make_twin() if make_twin is not None else None
+    if twin is not None:
+        sets.append((twin[0], twin[1]))
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    last = {"computed": None, "downloaded": None}
+    last = [{"computed": None, "downloaded": None} for _ in sets]
+    count = [0]
 
     def one():
+        b = count[0] % len(sets)
+        count[0] += 1
+        w, run = sets[b]
         ev_in, ev_comp, ev_out = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
-        if last["computed"] is not None:
-            s_in.wait_event(last["computed"])          # the previous step has read its inputs
+        if last[b]["computed"] is not None:
+            s_in.wait_event(last[b]["computed"])       # this set's previous step has read its inputs
         with torch.cuda.stream(s_in):
-            for h, d in zip(host_in, dev_in):
+            for h, d in zip(host_in, w.step_inputs):
                 d.copy_(h, non_blocking=True)
             ev_in.record(s_in)
         stream.wait_event(ev_in)
-        if last["downloaded"] is not None:
-            stream.wait_event(last["downloaded"])      # the previous outputs are on the host
-        run_step()
+        if last[b]["downloaded"] is not None:
+            stream.wait_event(last[b]["downloaded"])   # this set's previous outputs are on the host
+        run()
         ev_comp.record(stream)
         s_out.wait_event(ev_comp)
         with torch.cuda.stream(s_out):
-            for h, d in zip(host_out, outs):
+            for h, d in zip(host_out, w.outputs):
                 h.copy_(d, non_blocking=True)
             ev_out.record(s_out)
-        last["computed"], last["downloaded"] = ev_comp, ev_out
+        last[b]["computed"], last[b]["downloaded"] = ev_comp, ev_out
 
-    one()
+    for _ in sets:
+        one()
     torch.cuda.synchronize()
     barrier(ws)
     e0 = torch.cuda.Event(enable_timing=True)
@@ -590,7 +614,8 @@ def run_e2e(args, wl, stream, ws, run_step):
     s_in.wait_event(e0)                                # no upload starts before the timer
     for _ in range(steps):
         one()
-    stream.wait_event(last["downloaded"])
+    for l in last:
+        stream.wait_event(l["downloaded"])
     e1.record(stream)
     e1.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), ws)
@@ -598,7 +623,7 @@ def run_e2e(args, wl, stream, ws, run_step):
     tokens = wl.counts["tokens"] * len(wl.groups)
     return {"value": round(tokens * ws * steps / (ms / 1e3), 1), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 3)}
+            "ms_per_step": round(ms / steps, 3), "device_buffer_sets": len(sets)}
 
 
 def run_reference(args, ws, rank):
