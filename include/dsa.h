@@ -178,6 +178,12 @@ dsa_status dsa_sparse_mla_attn(const void* q, const dsa_cache_view* kv, const in
  *   q_pos0: position of prefill query row 0 (ignored for paged caches)
  *   q_rows_per_idx_row: 1 in prefill, 1 + d in decode with d MTP draft rows
  *   q[l] [n_idx_rows * q_rows_per_idx_row, 64, 576] bf16, kv[l] dim 576, out[l], lse[l]
+ *   workspace: at least dsa_group_workspace_bytes(a) bytes of device memory: e4m3 copies of
+ *              the indexer inputs (when quantised here), the scores of one chunk of query rows
+ *              (rows x causal length <= max(64 MB, 2,048 x longest row x 4 B), at most 1 GB),
+ *              the Top-k scratch and the split-KV partials of the attention.
+ * The call allocates nothing and only enqueues kernels and memsets on `stream`, so once a
+ * first call has set the device up it may be captured into a CUDA graph and replayed.
  */
 #define DSA_GROUP_MAX_LAYERS 4
 typedef struct {

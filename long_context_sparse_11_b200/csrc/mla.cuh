@@ -29,7 +29,7 @@
 // logits and folded into P^T).
 //
 // Warps 0..SM_WARPS-1: softmax / output (warp w: lane quadrant w%4, HPW heads from HPW*(w/4)),
-// and on the FP8 path part of the gather; the next 7 warps: query rows and the KV gather; the
+// and on the FP8 path part of the gather; the next GA_WARPS (7) warps: query rows and the KV gather; the
 // last warp: TMEM owner + MMA issuer.
 #pragma once
 #include <cuda_fp16.h>
