@@ -298,8 +298,8 @@ __global__ void __launch_bounds__(SEG_THREADS) topk_seg_filter_kernel(const floa
   int32_t* cnt = ws.counters + static_cast<int64_t>(r) * 4;
   uint32_t* ck = ws.cand_key + static_cast<int64_t>(r) * ws.gcap;
   int32_t* ci = ws.cand_idx + static_cast<int64_t>(r) * ws.gcap;
-  for (int32_t i = beg + t; i < end; i += SEG_THREADS) {
-    const uint32_t key = f32_key(row[i]);
+  auto visit = [&](float f, int32_t i) {
+    const uint32_t key = f32_key(f);
     const uint32_t d = key >> 20;
     if (d > T || (take_eq && d == T)) {
       const int32_t p = atomicAdd(&s_cnt[0], 1);
@@ -322,7 +322,32 @@ __global__ void __launch_bounds__(SEG_THREADS) topk_seg_filter_kernel(const floa
         }
       }
     }
+  };
+  // 16-byte loads, two in flight per thread (segments start at multiples of 4 and rows are
+  // 16-byte aligned), then the unaligned tail one by one
+  const int32_t end4 = beg + ((end - beg) & ~3);
+  int32_t i = beg + t * 4;
+  for (; i + SEG_THREADS * 4 < end4; i += SEG_THREADS * 8) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(row + i));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(row + i + SEG_THREADS * 4));
+    visit(a.x, i);
+    visit(a.y, i + 1);
+    visit(a.z, i + 2);
+    visit(a.w, i + 3);
+    const int32_t j = i + SEG_THREADS * 4;
+    visit(b.x, j);
+    visit(b.y, j + 1);
+    visit(b.z, j + 2);
+    visit(b.w, j + 3);
   }
+  if (i < end4) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(row + i));
+    visit(a.x, i);
+    visit(a.y, i + 1);
+    visit(a.z, i + 2);
+    visit(a.w, i + 3);
+  }
+  for (int32_t u = end4 + t; u < end; u += SEG_THREADS) visit(row[u], u);
   __syncthreads();
   const int32_t n_sel = min(s_cnt[0], SEL_BUF), n_cand = min(s_cnt[1], CAND_BUF);
   if (t == 0) {
