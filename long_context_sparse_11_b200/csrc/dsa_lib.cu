@@ -332,7 +332,7 @@ size_t mla_ws_bytes(int32_t n_q, int32_t k, int sms) {
 
 dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* idx, int32_t n_q, int32_t rpi,
                       int32_t k, float softmax_scale, void* out, float* lse, void* ws, size_t ws_bytes,
-                      cudaStream_t st) {
+                      cudaStream_t st, int64_t valid0 = -1) {
   DeviceState* ds = nullptr;
   DSA_TRY(device_state(&ds));
   if (n_q == 0) return DSA_OK;
@@ -357,6 +357,7 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
   p.status = ds->status;
   p.wait_ns = static_cast<uint64_t>(g_wait_ns);
   p.n_split = mla_splits(n_q, k, ds->sms);
+  p.valid0 = valid0;
   if (p.n_split > 1) {
     const size_t need = mla_ws_bytes(n_q, k, ds->sms);
     if (!ws || ws_bytes < need) return fail(DSA_ERR_WORKSPACE, "sparse MLA needs %zu workspace bytes", need);
@@ -728,10 +729,13 @@ dsa_status indexshare_group_forward(const dsa_group_args* a, dsa_index_handle* h
   }
   trace(ev, 1, st);
   const int32_t nq = n * a->q_rows_per_idx_row;
+  // indices computed by this call for a dense causal prefill: row i holds its min(k, q_pos0 + i + 1)
+  // valid entries first, so the attention skips the tiles past them
+  const int64_t valid0 = (!reuse_only && !a->idx_keys.block_table) ? static_cast<int64_t>(a->q_pos0) + 1 : -1;
   for (int l = 0; l < a->n_layers; ++l) {
     trace(ev, 2 + 2 * l, st);
     DSA_TRY(launch_mla(a->q[l], &a->kv[l], h->idx, nq, a->q_rows_per_idx_row, a->k, a->softmax_scale, a->out[l],
-                       a->lse[l], ws + g.off_mla, g.total - g.off_mla, st));
+                       a->lse[l], ws + g.off_mla, g.total - g.off_mla, st, valid0));
     trace(ev, 3 + 2 * l, st);
   }
   return DSA_OK;

@@ -102,6 +102,8 @@ struct Params {
   int32_t rows_per_idx;
   int32_t k;
   int32_t n_split;
+  int64_t valid0;            // >= 0: idx row i holds its valid entries first, min(k, valid0 + i) of
+                             // them (causal prefill); tiles past them are skipped.  < 0: k
   int32_t max_pages;
   int32_t n_pages;
   float scale_log2;          // softmax_scale * log2(e)
@@ -223,8 +225,13 @@ __device__ __forceinline__ Item make_item(const Params& p, int32_t item) {
   it.irow = it.row / p.rows_per_idx;
   const int32_t all = (p.k + TILE - 1) / TILE;
   const int32_t tps = (all + p.n_split - 1) / p.n_split;
+  int32_t used = all;
+  if (p.valid0 >= 0) {
+    const int64_t v = min(static_cast<int64_t>(p.k), p.valid0 + it.irow);
+    used = static_cast<int32_t>((max(v, static_cast<int64_t>(0)) + TILE - 1) / TILE);
+  }
   it.j0 = it.split * tps;
-  it.n_tiles = max(0, min(it.j0 + tps, all) - it.j0);
+  it.n_tiles = max(0, min(it.j0 + tps, used) - it.j0);
   return it;
 }
 
