@@ -94,14 +94,17 @@ struct Params {
   const int32_t* idx;        // [n_idx_rows, k]
   uint16_t* out;             // [n_q,64,512] bf16
   float* lse;                // [n_q,64] or null
-  float* part_o;             // split partials [n_q*n_split,64,512] fp32
+  float* part_o;             // partials [n_q*n_split,64,512] fp32 (row r, slot s at r*n_split+s)
   float* part_ml;            // [n_q*n_split,2,64] (m in log2 units, l)
   int64_t row_stride;        // elements (dense)
   int64_t n_tokens;
   int32_t n_q;
   int32_t rows_per_idx;
   int32_t k;
-  int32_t n_split;
+  int32_t n_split;          // slots per row (equal splits, or at most this many stream-K fragments)
+  int32_t stream_k;          // 1: CTA c takes the contiguous tile range [c*G/grid, (c+1)*G/grid) of the
+                             // n_q x tiles_per_row tiles in row order; rows cut by a range boundary
+                             // leave partials per fragment, whole rows are written directly
   int64_t valid0;            // >= 0: idx row i holds its valid entries first, min(k, valid0 + i) of
                              // them (causal prefill); tiles past them are skipped.  < 0: k
   int32_t max_pages;
@@ -214,14 +217,60 @@ __device__ __forceinline__ int64_t kv_row(const Params& p, int32_t seq, int32_t 
   return static_cast<int64_t>(pg) * 64 + (v & 63);
 }
 
-// Work item -> (query row, idx row, first tile, number of tiles).
+// Work item -> (query row, idx row, first tile, number of tiles, partial slot, written directly).
 struct Item {
   int32_t row, irow, j0, n_tiles, split;
+  bool direct;
 };
+
+// Stream-K: the CTA owning global tile g of G tiles split over `grid` CTAs.
+__host__ __device__ __forceinline__ int64_t sk_owner(int64_t g, int64_t G, int64_t grid) {
+  return ((g + 1) * grid - 1) / G;
+}
+
+// The CTA's sequence of items: strided (row, split) items, or its stream-K tile range.
+struct WorkIter {
+  int64_t a, b;
+};
+__device__ __forceinline__ WorkIter work_begin(const Params& p) {
+  WorkIter w;
+  if (p.stream_k) {
+    const int64_t G = static_cast<int64_t>(p.n_q) * ((p.k + TILE - 1) / TILE);
+    w.a = static_cast<int64_t>(blockIdx.x) * G / gridDim.x;
+    w.b = static_cast<int64_t>(blockIdx.x + 1) * G / gridDim.x;
+  } else {
+    w.a = blockIdx.x;
+    w.b = static_cast<int64_t>(p.n_q) * p.n_split;
+  }
+  return w;
+}
+
+__device__ __forceinline__ Item make_item(const Params& p, int32_t item);
+
+__device__ __forceinline__ bool work_next(const Params& p, WorkIter& w, Item& it) {
+  if (w.a >= w.b) return false;
+  if (!p.stream_k) {
+    it = make_item(p, static_cast<int32_t>(w.a));
+    w.a += gridDim.x;
+    return true;
+  }
+  const int32_t tpr = (p.k + TILE - 1) / TILE;
+  const int64_t G = static_cast<int64_t>(p.n_q) * tpr;
+  it.row = static_cast<int32_t>(w.a / tpr);
+  it.irow = it.row / p.rows_per_idx;
+  it.j0 = static_cast<int32_t>(w.a % tpr);
+  it.n_tiles = static_cast<int32_t>(min(static_cast<int64_t>(tpr - it.j0), w.b - w.a));
+  it.direct = it.j0 == 0 && it.n_tiles == tpr;
+  it.split = static_cast<int32_t>(blockIdx.x - sk_owner(static_cast<int64_t>(it.row) * tpr, G, gridDim.x));
+  w.a += it.n_tiles;
+  return true;
+}
+
 __device__ __forceinline__ Item make_item(const Params& p, int32_t item) {
   Item it;
   it.row = item / p.n_split;
   it.split = item % p.n_split;
+  it.direct = p.n_split == 1;
   it.irow = it.row / p.rows_per_idx;
   const int32_t all = (p.k + TILE - 1) / TILE;
   const int32_t tps = (all + p.n_split - 1) / p.n_split;
@@ -276,7 +325,6 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
   float* l_tot = reinterpret_cast<float*>(misc + M_LTOT);
   float* red = reinterpret_cast<float*>(misc + M_RED);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int32_t n_items = p.n_q * p.n_split;
   constexpr bool SM_GATHER = sm_gather<PAGED>();
   constexpr int NG = n_gather<PAGED>();
 
@@ -391,8 +439,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
     const int gq = threadIdx.x - SM_THREADS;  // query-row loader index
     uint32_t gtile = 0;
     bool ok = true;
-    for (int32_t item = blockIdx.x, it_n = 0; item < n_items && ok; item += gridDim.x, ++it_n) {
-      const Item it = make_item(p, item);
+    WorkIter wk = work_begin(p);
+    Item it;
+    for (int32_t it_n = 0; ok && work_next(p, wk, it); ++it_n) {
       // ---- query row -> 9 K-major sub-tiles (bf16 copy, or bf16 -> f16 for the FP8 cache path)
       if (!mbar_wait(bar(B_QEMPTY), (it_n & 1) ^ 1, abort_flag, p.status, p.wait_ns)) break;
       const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q + static_cast<int64_t>(it.row) * 64 * 576);
@@ -445,8 +494,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
       constexpr uint32_t ID_PV = make_idesc(FMT, FMT, 1, 1, 128, 64);
       uint32_t gtile = 0;
       bool ok = true;
-      for (int32_t item = blockIdx.x, it_n = 0; item < n_items && ok; item += gridDim.x, ++it_n) {
-        const Item it = make_item(p, item);
+      WorkIter wk = work_begin(p);
+      Item it;
+      for (int32_t it_n = 0; ok && work_next(p, wk, it); ++it_n) {
         if (!mbar_wait(bar(B_QFULL), it_n & 1, abort_flag, p.status, p.wait_ns)) break;
         fence_async_smem();
         tc_fence_after();
@@ -497,8 +547,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
     const bool head_lane = lane < HPW;                // lanes that own one of the warp's heads
     uint32_t gtile = 0;
     bool ok = true;
-    for (int32_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const Item it = make_item(p, item);
+    WorkIter wk = work_begin(p);
+    Item it;
+    while (ok && work_next(p, wk, it)) {
       const int32_t seq_len = PAGED ? p.seq_lens[it.irow] : 0;
       const int32_t* idx_row = p.idx + static_cast<int64_t>(it.irow) * p.k;
       if (quad == 0 && head_lane) m_run[hcol + lane] = -INFINITY;
@@ -631,7 +682,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         l_tot[h] = red[h] + red[64 + h] + red[128 + h] + red[192 + h];
       }
       named_bar(1, SM_THREADS);
-      if (p.n_split == 1) {
+      if (it.direct) {
         uint16_t* orow = p.out + static_cast<int64_t>(it.row) * 64 * 512;
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
@@ -688,19 +739,29 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
   if (warp == MMA_WARP) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-// Combine split-KV partials: one CTA of 128 threads per (row, head), 4 dims per thread.
+// Combine split-KV partials: one CTA of 128 threads per (row, head), 4 dims per thread.  Equal
+// splits: n_split slots per row.  Stream-K (grid > 0): the row's fragments came from CTAs
+// sk_owner(first tile) .. sk_owner(last tile); a row inside one CTA was written directly.
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part_o,
                                                       const float* __restrict__ part_ml, int32_t n_split,
-                                                      uint16_t* __restrict__ out, float* __restrict__ lse) {
+                                                      uint16_t* __restrict__ out, float* __restrict__ lse,
+                                                      int32_t tiles_per_row, int64_t sk_tiles, int32_t sk_grid) {
   const int32_t row = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
+  int32_t n_slots = n_split;
+  if (sk_grid > 0) {
+    const int64_t g0 = static_cast<int64_t>(row) * tiles_per_row;
+    n_slots = static_cast<int32_t>(sk_owner(g0 + tiles_per_row - 1, sk_tiles, sk_grid) -
+                                   sk_owner(g0, sk_tiles, sk_grid) + 1);
+    if (n_slots == 1) return;
+  }
   float M = -INFINITY;
-  for (int s = 0; s < n_split; ++s) {
+  for (int s = 0; s < n_slots; ++s) {
     const int64_t pr = static_cast<int64_t>(row) * n_split + s;
     if (part_ml[pr * 128 + 64 + h] > 0.f) M = fmaxf(M, part_ml[pr * 128 + h]);
   }
   float L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < n_split; ++s) {
+  for (int s = 0; s < n_slots; ++s) {
     const int64_t pr = static_cast<int64_t>(row) * n_split + s;
     const float l = part_ml[pr * 128 + 64 + h];
     if (!(l > 0.f)) continue;
