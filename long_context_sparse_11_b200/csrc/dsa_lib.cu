@@ -110,10 +110,16 @@ dsa_status device_state(DeviceState** out) {
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             idx::Cfg<true, true>::SMEM_BYTES),
                        "smem attr"));
-    DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<false>,
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<false, false>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES),
                        "smem attr"));
-    DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<true>,
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<true, false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES),
+                       "smem attr"));
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<false, true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES),
+                       "smem attr"));
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<true, true>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES),
                        "smem attr"));
     DSA_TRY(cuda_check(cudaFuncSetAttribute(topk::topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -400,10 +406,15 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
   const unsigned grid = sk.on ? static_cast<unsigned>(sk.grid)
                               : static_cast<unsigned>(std::min<int64_t>(static_cast<int64_t>(n_q) * p.n_split,
                                                                         static_cast<int64_t>(ds->sms)));
-  if (paged)
-    mla::sparse_mla_kernel<true><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
-  else
-    mla::sparse_mla_kernel<false><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
+  if (paged && sk.on) {
+    mla::sparse_mla_kernel<true, true><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
+  } else if (paged) {
+    mla::sparse_mla_kernel<true, false><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
+  } else if (sk.on) {
+    mla::sparse_mla_kernel<false, true><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
+  } else {
+    mla::sparse_mla_kernel<false, false><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
+  }
   count_launch();
   DSA_TRY(cuda_check(cudaGetLastError(), "sparse MLA launch"));
   if (p.n_split > 1) {

@@ -102,7 +102,7 @@ struct Params {
   int32_t rows_per_idx;
   int32_t k;
   int32_t n_split;          // slots per row (equal splits, or at most this many stream-K fragments)
-  int32_t stream_k;          // 1: CTA c takes the contiguous tile range [c*G/grid, (c+1)*G/grid) of the
+  int32_t stream_k;          // (kernels instantiated with SK) 1: CTA c takes the contiguous tile range [c*G/grid, (c+1)*G/grid) of the
                              // n_q x tiles_per_row tiles in row order; rows cut by a range boundary
                              // leave partials per fragment, whole rows are written directly
   int64_t valid0;            // >= 0: idx row i holds its valid entries first, min(k, valid0 + i) of
@@ -232,9 +232,10 @@ __host__ __device__ __forceinline__ int64_t sk_owner(int64_t g, int64_t G, int64
 struct WorkIter {
   int64_t a, b;
 };
+template <bool SK>
 __device__ __forceinline__ WorkIter work_begin(const Params& p) {
   WorkIter w;
-  if (p.stream_k) {
+  if constexpr (SK) {
     const int64_t G = static_cast<int64_t>(p.n_q) * ((p.k + TILE - 1) / TILE);
     w.a = static_cast<int64_t>(blockIdx.x) * G / gridDim.x;
     w.b = static_cast<int64_t>(blockIdx.x + 1) * G / gridDim.x;
@@ -247,9 +248,10 @@ __device__ __forceinline__ WorkIter work_begin(const Params& p) {
 
 __device__ __forceinline__ Item make_item(const Params& p, int32_t item);
 
+template <bool SK>
 __device__ __forceinline__ bool work_next(const Params& p, WorkIter& w, Item& it) {
   if (w.a >= w.b) return false;
-  if (!p.stream_k) {
+  if constexpr (!SK) {
     it = make_item(p, static_cast<int32_t>(w.a));
     w.a += gridDim.x;
     return true;
@@ -308,7 +310,7 @@ __device__ __forceinline__ void e4m3x16_to_f16(uint4 raw, uint4& o0, uint4& o1) 
   o1 = make_uint4(r[4], r[5], r[6], r[7]);
 }
 
-template <bool PAGED>
+template <bool PAGED, bool SK>
 __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -439,9 +441,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
     const int gq = threadIdx.x - SM_THREADS;  // query-row loader index
     uint32_t gtile = 0;
     bool ok = true;
-    WorkIter wk = work_begin(p);
+    WorkIter wk = work_begin<SK>(p);
     Item it;
-    for (int32_t it_n = 0; ok && work_next(p, wk, it); ++it_n) {
+    for (int32_t it_n = 0; ok && work_next<SK>(p, wk, it); ++it_n) {
       // ---- query row -> 9 K-major sub-tiles (bf16 copy, or bf16 -> f16 for the FP8 cache path)
       if (!mbar_wait(bar(B_QEMPTY), (it_n & 1) ^ 1, abort_flag, p.status, p.wait_ns)) break;
       const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q + static_cast<int64_t>(it.row) * 64 * 576);
@@ -494,9 +496,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
       constexpr uint32_t ID_PV = make_idesc(FMT, FMT, 1, 1, 128, 64);
       uint32_t gtile = 0;
       bool ok = true;
-      WorkIter wk = work_begin(p);
+      WorkIter wk = work_begin<SK>(p);
       Item it;
-      for (int32_t it_n = 0; ok && work_next(p, wk, it); ++it_n) {
+      for (int32_t it_n = 0; ok && work_next<SK>(p, wk, it); ++it_n) {
         if (!mbar_wait(bar(B_QFULL), it_n & 1, abort_flag, p.status, p.wait_ns)) break;
         fence_async_smem();
         tc_fence_after();
@@ -547,9 +549,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
     const bool head_lane = lane < HPW;                // lanes that own one of the warp's heads
     uint32_t gtile = 0;
     bool ok = true;
-    WorkIter wk = work_begin(p);
+    WorkIter wk = work_begin<SK>(p);
     Item it;
-    while (ok && work_next(p, wk, it)) {
+    while (ok && work_next<SK>(p, wk, it)) {
       const int32_t seq_len = PAGED ? p.seq_lens[it.irow] : 0;
       const int32_t* idx_row = p.idx + static_cast<int64_t>(it.irow) * p.k;
       if (quad == 0 && head_lane) m_run[hcol + lane] = -INFINITY;
