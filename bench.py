@@ -399,7 +399,6 @@ def run_ours(args, ws, rank, local):
     for _ in range(args.warmup):
         step(False)
     dsa.sync_status()
-    barrier(ws)
     torch.cuda.synchronize()
     n0 = lib.dsa_launch_count()
     step(False)
@@ -444,15 +443,18 @@ def run_ours(args, ws, rank, local):
         return out
 
     mla_ms, idx_ms = [], []
+    torch.cuda.synchronize()
+    barrier(ws)                                             # all ranks start the timed steps together
     with ClockSampler(gpu_smi_id(local)) as clk:
         # eager steps carry the library's phase events; graph replays are timed on their own and
         # the phase split comes from as many eager steps run afterwards
         t_steps = timed_steps(args.steps, traced=graph is None)
+    torch.cuda.synchronize()
+    barrier(ws)
     if graph is not None:
         timed_steps(args.steps, traced=True)
-    torch.cuda.synchronize()
+        torch.cuda.synchronize()
     launches = launches_per_step * args.steps
-    barrier(ws)
     dsa.sync_status()
     total_ms = max_over_ranks(sum(t_steps), ws)
     ms_per_step = total_ms / args.steps
