@@ -254,6 +254,17 @@ class ClockSampler:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
             self.lines = [l for l in out.splitlines() if l.strip()]
+        self.after = False
+        if self.proc is not None and not self.lines:
+            # a timed region shorter than one sampling period: one reading right after it
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=10).stdout
+                self.lines = [l for l in out.splitlines() if l.strip()]
+                self.after = bool(self.lines)
+            except (OSError, subprocess.TimeoutExpired):
+                pass
 
     def summary(self):
         sm, mx, reasons = [], None, set()
@@ -270,8 +281,11 @@ class ClockSampler:
             for n, v in zip(names, f[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+               "samples": 0 if getattr(self, "after", False) else len(sm)}
+        if getattr(self, "after", False):
+            out["read_after_timed_region"] = True   # the region was shorter than the 100 ms period
+        return out
 
 
 def gpu_smi_id(dev_index):
