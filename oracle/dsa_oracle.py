@@ -21,7 +21,10 @@ reading, listed once here and used consistently:
 R1  Indexer score: I[t,s] = sum_h w[t,h] * max(0, q[t,h,:] . k[s,:]) over 32 heads of 128
     dims (a lightweight indexer that scores each history token per query, [forum]
     "IndexShare：省掉3/4的索引计算"; 32 indexer heads, [ailearn] architecture card).  No
-    global constant: a positive constant leaves the Top-k unchanged.
+    global constant: a positive constant leaves the Top-k unchanged.  The pages print no
+    formula and no value for it, so indexer_scores is parity unpinned by the pages: its
+    tests pin it to this definition (closed forms on unit vectors, invariances), not to a
+    printed number.
 R2  Causal candidates include the query itself: s <= t (prefill); s < N_b in decode,
     where N_b counts the current token.
 R3  Top-k keeps the k largest scores; equal scores go to the lower index; with fewer than
