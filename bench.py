@@ -30,10 +30,10 @@ sys.path.insert(0, ROOT)
 METRIC = "query tokens/s per IndexShare group"
 UNIT = "query tokens/s"
 
-# sparse_mla_kernel<bf16>, L=8,192 prefill launch (8,192 query rows): ncu measured 681.4 MB read
-# + 504.8 MB written = 144,799 B per query row (queries 73,728 B in, outputs 65,536 B out, the
+# sparse_mla_kernel<bf16>, L=8,192 prefill launch (8,192 query rows): ncu measured 672.8 MB read
+# + 510.4 MB written = 144,436 B per query row (queries 73,728 B in, outputs 65,536 B out, the
 # rest index rows and the latent rows' first touch).
-MLA_DRAM_BYTES_PER_ROW_BF16 = (681.366528e6 + 504.834048e6) / 8192
+MLA_DRAM_BYTES_PER_ROW_BF16 = (672.798720e6 + 510.417920e6) / 8192
 
 
 
