@@ -23,6 +23,22 @@ namespace idx {
 constexpr int BLOCK_KEYS = 128;
 constexpr int UNIT_TILES = 32;  // key tiles per work unit (default; decode may use fewer)
 
+// ReLU split between two pipes.  max(x, 0) runs on the ALU pipe, which the epilogue saturates
+// first; for P of the 16 head pairs the epilogue instead forms x + |x| = 2 max(x, 0) with one
+// add on the FMA pipe and the staged weight of those heads is halved, so w * max(x, 0) is
+// reproduced exactly (0.5 w * 2x = w * x for every finite accumulator x).  The P pairs are
+// spread evenly over the 16.
+#ifndef DSA_IDX_RELU_FMA_PAIRS_BF16
+#define DSA_IDX_RELU_FMA_PAIRS_BF16 8
+#endif
+#ifndef DSA_IDX_RELU_FMA_PAIRS_E4M3
+#define DSA_IDX_RELU_FMA_PAIRS_E4M3 8
+#endif
+template <int P>
+__host__ __device__ constexpr bool relu_on_fma(int pair) {
+  return ((pair + 1) * P) / 16 != (pair * P) / 16;
+}
+
 template <bool FP8, bool PAGED>
 struct Cfg {
   static constexpr int NQ = PAGED ? 1 : 8;        // queries per accumulator
@@ -34,6 +50,7 @@ struct Cfg {
   static constexpr int KSTEPS = FP8 ? 4 : 8;
   static constexpr int STAGES = FP8 ? 4 : 2;
   static constexpr int EPI_WARPS = PAGED ? 4 : 16;
+  static constexpr int RELU_FMA_PAIRS = FP8 ? DSA_IDX_RELU_FMA_PAIRS_E4M3 : DSA_IDX_RELU_FMA_PAIRS_BF16;
   static constexpr int THREADS = 64 + EPI_WARPS * 32;
   static constexpr int Q_HALF_BYTES = N * 128;    // one K half of one query group
   static constexpr int Q_BYTES = NGROUP * KH * Q_HALF_BYTES;
@@ -139,6 +156,7 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
       if (row < p.n_q) {
         v = p.w[static_cast<int64_t>(row) * 32 + h];
         if (FP8) v *= p.q_scale[static_cast<int64_t>(row) * 32 + h];
+        if (relu_on_fma<C::RELU_FMA_PAIRS>(h >> 1)) v *= 0.5f;
       }
       w_s[i] = v;
     }
@@ -269,10 +287,14 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
 #pragma unroll
           for (int h4 = 0; h4 < 8; ++h4) {
             const float4 ww = wv[h4];
-            ffma2(a0, a1, ww.x, ww.y, fmaxf(__uint_as_float(x[4 * h4]), 0.f),
-                  fmaxf(__uint_as_float(x[4 * h4 + 1]), 0.f));
-            ffma2(a0, a1, ww.z, ww.w, fmaxf(__uint_as_float(x[4 * h4 + 2]), 0.f),
-                  fmaxf(__uint_as_float(x[4 * h4 + 3]), 0.f));
+            float r[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float v = __uint_as_float(x[4 * h4 + u]);
+              r[u] = relu_on_fma<C::RELU_FMA_PAIRS>(2 * h4 + u / 2) ? v + fabsf(v) : fmaxf(v, 0.f);
+            }
+            ffma2(a0, a1, ww.x, ww.y, r[0], r[1]);
+            ffma2(a0, a1, ww.z, ww.w, r[2], r[3]);
           }
           float acc = a0 + a1;
           if (FP8) acc *= sk;
