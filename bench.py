@@ -44,6 +44,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--workload", default="prefill_32k",
                    choices=["tiny_prefill", "prefill_32k", "prefill_128k_fp8", "decode_b32_mtp4", "decode_b32_d0",
+                            "decode_b32_mtp4_verify",
                             "decode_1m_mtp5"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
@@ -110,7 +111,8 @@ def workload_config(name, seq_len=None):
     if name.startswith("decode"):
         cfg = {"workload": name, "batch": spec.batch, "context": f"U[{spec.ctx_lo},{spec.ctx_hi}]",
                "rows_per_seq": spec.rows_per_seq, "k": spec.k, "layers": spec.n_layers,
-               "cache": "paged e4m3 (64-token pages), device-resident across steps", "indexer": "e4m3"}
+               "cache": "paged e4m3 (64-token pages), device-resident across steps", "indexer": "e4m3",
+               "topk": "one per query row" if spec.topk_per_row else "row 0's, reused by the draft rows"}
         if spec.n_layers > 4:
             cfg["schedule"] = "Full at layers 0, 1, 2+4g; 21 groups per step"
         return spec, cfg
@@ -131,10 +133,13 @@ def algorithmic_counts(spec, ctx=None):
     ctx = np.asarray(ctx)
     R = spec.rows_per_seq
     sel = float(np.minimum(ctx, spec.k).sum())
-    return {"tokens": len(ctx) * R, "indexer_flops": 8192.0 * float(ctx.sum()),
+    # per-row Top-k: R indexer queries per sequence over the same keys (the keys' bytes are still
+    # needed once), and up to R distinct selections per sequence to gather
+    scored = R if spec.topk_per_row else 1
+    return {"tokens": len(ctx) * R, "indexer_flops": 8192.0 * float(ctx.sum()) * scored,
             "mla_flops_per_layer": 139264.0 * sel * R, "mla_rows": len(ctx) * R,
             "indexer_bytes": 132.0 * float(ctx.sum()),
-            "mla_bytes_per_layer": sel * 580.0 + len(ctx) * R * 64 * (576 + 512) * 2.0}
+            "mla_bytes_per_layer": sel * scored * 580.0 + len(ctx) * R * 64 * (576 + 512) * 2.0}
 
 
 class Workload:
@@ -151,15 +156,18 @@ class Workload:
             self.inp = inp
             ctx_d = torch.from_numpy(inp["ctx"].astype("int32")).to(dev)
             bt_d = torch.from_numpy(inp["block_table"]).to(dev)
-            kvs = [dsa.paged_view(inp["KV"][l], inp["KV_scale"][l], bt_d, ctx_d) for l in range(spec.n_layers)]
+            # per-row Top-k: every query row is its own entry of the views (same pages, same length)
+            rows = spec.rows_per_seq if spec.topk_per_row else 1
+            kvs = [dsa.paged_view(inp["KV"][l], inp["KV_scale"][l], bt_d, ctx_d, rows_per_seq=rows)
+                   for l in range(spec.n_layers)]
             fulls = [l for l in range(spec.n_layers) if dsa.layer_is_full(l)] if spec.n_layers > 4 else [0]
             ends = fulls[1:] + [spec.n_layers]
             for f, e in zip(fulls, ends):
                 ind = inp if f == 0 else make_decode_indexer(spec, f, inp["n_pages"], len(inp["ctx"]), dev)
-                keys = dsa.paged_view(ind["idx_keys"], ind["idx_key_scale"], bt_d, ctx_d)
+                keys = dsa.paged_view(ind["idx_keys"], ind["idx_key_scale"], bt_d, ctx_d, rows_per_seq=rows)
                 g = dsa.IndexShareGroup(ind["q_idx"], ind["w"], keys, spec.k, inp["Q"][f:e], kvs[f:e],
                                         inp["softmax_scale"], indexer_dtype=dsa.DSA_E4M3,
-                                        q_rows_per_idx_row=spec.rows_per_seq, first_layer=f)
+                                        q_rows_per_idx_row=spec.rows_per_seq // rows, first_layer=f)
                 self.groups.append(g)
                 self.layers_per_group.append(e - f)
                 # a decode step's new inputs: the indexer query and weights, the MLA query rows
@@ -324,10 +332,11 @@ def oracle_rows_per_second(spec, name, inp, budget_s, seed_rows=0):
                 "idx_keys": inp["idx_keys"].cpu().numpy(), "idx_key_scale": inp["idx_key_scale"].cpu().numpy(),
                 "Q": [host_bits(q) for q in inp["Q"][:nl]], "KV": [x.cpu().numpy() for x in inp["KV"][:nl]],
                 "KV_scale": [x.cpu().numpy() for x in inp["KV_scale"][:nl]]}
+        policy = O.group_decode_per_row if spec.topk_per_row else O.group_decode
         order = list(np.random.default_rng(seed_rows).permutation(len(inp["ctx"])))
         done, t0 = 0, time.perf_counter()
         while order and time.perf_counter() - t0 < budget_s:
-            O.group_decode(host, seqs=[order.pop()])
+            policy(host, seqs=[order.pop()])
             done += spec.rows_per_seq
         el = time.perf_counter() - t0
         return done / el, (f"{done // spec.rows_per_seq} whole sequences (all {spec.rows_per_seq} rows, indexer, "

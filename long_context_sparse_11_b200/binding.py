@@ -126,11 +126,19 @@ def dense_view(data, scale=None) -> CacheView:
     return v
 
 
-def paged_view(pool, scale, block_table, seq_lens) -> CacheView:
+def paged_view(pool, scale, block_table, seq_lens, rows_per_seq: int = 1) -> CacheView:
     """Paged e4m3 cache: pool [n_pages,64,dim] uint8, scale [n_pages,64] fp32,
-    block_table [B,max_pages] int32, seq_lens [B] int32 (all on the device)."""
+    block_table [B,max_pages] int32, seq_lens [B] int32 (all on the device).
+
+    rows_per_seq > 1 presents each sequence as that many consecutive entries sharing its pages
+    and length (the block-table rows and lengths are repeated once, here; the pages are not
+    copied): the view through which every MTP verification row is scored, selected and attended
+    as its own row, for a per-row Top-k instead of the reuse of row 0's."""
     n_pages, page, dim = pool.shape
-    assert page == 64
+    assert page == 64 and rows_per_seq >= 1
+    if rows_per_seq > 1:
+        block_table = block_table.repeat_interleave(rows_per_seq, dim=0).contiguous()
+        seq_lens = seq_lens.repeat_interleave(rows_per_seq).contiguous()
     v = CacheView(pool.data_ptr(), scale.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(), dim,
                   n_pages * 64, dim, DSA_E4M3, block_table.shape[1], block_table.shape[0])
     v._keep = (pool, scale, block_table, seq_lens)

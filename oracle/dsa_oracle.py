@@ -40,6 +40,11 @@ R6  IndexShare: the Full layer's indices are passed unchanged to the next 3 Shar
 R7  MTP: the first draft step's Top-k is reused by later steps and drafts add no KV
     (KV Share) ([ailearn] MTP section; [forum] "MTP推测解码改进").  In one decode step
     the 1+d query rows of a sequence all use row 0's indices and the same cache.
+V1  MTP verification, the alternative to R7: each of the 1+d query rows of a sequence has its
+    own indexer query and head weights, scores the same N_b cached keys (drafts still add
+    no KV) and keeps its own Top-k, which that row's sparse MLA uses in every layer of the
+    group.  The pages describe only the reuse of R7 ([ailearn] MTP section); this policy
+    is what that reuse saves, so it is built to be compared against it.
 R8  78-layer schedule: Full at 0-based layers 0, 1 and 2 + 4g; the rest Shared, each
     reusing the preceding Full layer ([ailearn] "IndexShare：四层共用一次搜索结果").
 """
@@ -52,7 +57,7 @@ import numpy as np
 __all__ = [
     "bf16_to_f64", "e4m3_to_f64", "quantize_e4m3_rows", "indexer_scores", "topk_rows",
     "topk_row", "sparse_mla_row", "dense_causal_attention_row", "sparse_mla",
-    "group_prefill", "group_decode", "layer_schedule", "indexer_param_count",
+    "group_prefill", "group_decode", "group_decode_per_row", "layer_schedule", "indexer_param_count",
     "E4M3_MAX", "IDX_HEADS", "IDX_DIM", "MLA_HEADS", "D_QK", "D_V", "PAGE",
 ]
 
@@ -292,6 +297,40 @@ def group_decode(inp: dict, seqs=None, idx_override=None, layers=None):
             for r in range(R):
                 row = b * R + r
                 O[row], Ls[row] = sparse_mla_row(bf16_to_f64(inp["Q"][l][row]), kvrows, idx[b],
+                                                 inp["softmax_scale"])
+        outO.append(O)
+        outL.append(Ls)
+    return {"idx": idx, "O": outO, "lse": outL}
+
+
+def group_decode_per_row(inp: dict, seqs=None, layers=None):
+    """One IndexShare group in batched decode where every query row takes its own Top-k (V1).
+
+    inp holds q_idx [B*R,32,128] and w [B*R,32]: query row b*R + r scores sequence b's N_b
+    cached keys with its own e4m3-quantised indexer query, keeps its own Top-k, and attends
+    over those rows in every layer of the group."""
+    ctx, bt, k, R = inp["ctx"], inp["block_table"], inp["k"], inp["rows_per_seq"]
+    seqs = range(len(ctx)) if seqs is None else seqs
+    q8, sq = quantize_e4m3_rows(inp["q_idx"], IDX_DIM)
+    qv = e4m3_to_f64(q8) * sq.reshape(-1, IDX_HEADS, 1)
+    w = np.asarray(inp["w"], dtype=np.float64)
+    idx = {}
+    for b in seqs:
+        n = int(ctx[b])
+        keys = paged_rows(inp["idx_keys"], inp["idx_key_scale"], bt[b], n)
+        for r in range(R):
+            row = b * R + r
+            sc = indexer_scores(qv[row:row + 1], w[row:row + 1], keys, [n])[0]
+            idx[row] = topk_row(sc, n, k)
+    layers = range(len(inp["Q"])) if layers is None else layers
+    outO, outL = [], []
+    for l in layers:
+        O, Ls = {}, {}
+        for b in seqs:
+            kvrows = paged_rows(inp["KV"][l], inp["KV_scale"][l], bt[b], int(ctx[b]))
+            for r in range(R):
+                row = b * R + r
+                O[row], Ls[row] = sparse_mla_row(bf16_to_f64(inp["Q"][l][row]), kvrows, idx[row],
                                                  inp["softmax_scale"])
         outO.append(O)
         outL.append(Ls)

@@ -1,4 +1,4 @@
-"""Input recipes for the five workloads (seeded, synthetic; no method arithmetic here).
+"""Input recipes for the workloads (seeded, synthetic; no method arithmetic here).
 
 Workloads, named by what they are:
 
@@ -13,6 +13,10 @@ Workloads, named by what they are:
 * ``decode_b32_d0``   the same batch and caches as ``decode_b32_mtp4`` with one query row per
                       sequence (no draft rows): sparse MLA reads 580 B per selected key for 139,264
                       flops, so it is bound by memory rather than by the tensor cores.
+* ``decode_b32_mtp4_verify`` the batch, caches and MLA rows of ``decode_b32_mtp4``, but each of
+                      the 5 rows of a sequence has its own indexer query and head weights (row 0
+                      keeps the ``decode_b32_mtp4`` ones) and takes its own Top-k: the per-token
+                      selection for MTP verification rows, against the reuse of row 0's.
 * ``decode_1m_mtp5``  1 sequence of 1,048,576 tokens, 1 + 5 rows, 78-layer schedule.
 
 Stream ids keep every tensor independent: ``sub_seed(seed, layer, TENSOR_ID)``.
@@ -38,6 +42,7 @@ MLA_HEADS, D_QK, D_V = 64, 576, 512
 PAGE = 64
 
 T_QIDX, T_W, T_KIDX, T_Q, T_KV, T_PERM, T_CTX, T_KSCALE, T_KVSCALE = range(1, 10)
+T_QIDX_DRAFT, T_W_DRAFT = 10, 11   # indexer query and weights of draft rows (per-row Top-k only)
 
 
 @dataclass
@@ -66,6 +71,7 @@ class DecodeSpec:
     fixed_ctx: int | None = None
     softmax_scale: float = 1.0 / math.sqrt(D_QK)
     full_layers: list = field(default_factory=lambda: [0])
+    topk_per_row: bool = False    # every query row has its own indexer query and Top-k
 
 
 WORKLOADS = {
@@ -75,6 +81,8 @@ WORKLOADS = {
     "decode_b32_mtp4": DecodeSpec("decode_b32_mtp4", batch=32, ctx_lo=65536, ctx_hi=262144,
                                   rows_per_seq=5, seed=4),
     "decode_b32_d0": DecodeSpec("decode_b32_d0", batch=32, ctx_lo=65536, ctx_hi=262144, rows_per_seq=1, seed=4),
+    "decode_b32_mtp4_verify": DecodeSpec("decode_b32_mtp4_verify", batch=32, ctx_lo=65536, ctx_hi=262144,
+                                         rows_per_seq=5, seed=4, topk_per_row=True),
     "decode_1m_mtp5": DecodeSpec("decode_1m_mtp5", batch=1, ctx_lo=1 << 20, ctx_hi=1 << 20,
                                  rows_per_seq=6, seed=5, n_layers=78, fixed_ctx=1 << 20),
 }
@@ -97,6 +105,14 @@ def _f32(x, device):
         return np.asarray(x, dtype=np.float32)
     import torch
     return x.to(torch.float32)
+
+
+def _cat_rows(first, rest, shape):
+    """Row 0 of each sequence from `first` [B,...], rows 1.. from `rest` [B,R-1,...], flattened."""
+    if isinstance(first, np.ndarray):
+        return np.concatenate([first[:, None], rest], axis=1).reshape(shape)
+    import torch
+    return torch.cat([first[:, None], rest], dim=1).reshape(shape)
 
 
 def make_prefill(spec: PrefillSpec, L: int | None = None, device=None, layers=None) -> dict:
@@ -199,7 +215,9 @@ def make_decode_indexer(spec: DecodeSpec, layer: int, n_pages: int, batch: int, 
 def make_decode(spec: DecodeSpec, device=None, ctx=None, layers=None) -> dict:
     """Inputs of one decode step (batch of sequences with paged FP8 caches).
 
-    Layouts: q_idx [B,32,128] bf16 (row 0 of each sequence), w [B,32] fp32,
+    Layouts: q_idx [B,32,128] bf16 (row 0 of each sequence), w [B,32] fp32; with
+    ``topk_per_row`` q_idx [B*R,32,128] and w [B*R,32], row b*R the same as above and rows
+    b*R+1..b*R+R-1 from their own streams;
     idx_keys [P,64,128] e4m3 + idx_key_scale [P,64] fp32 (one pool per Full layer),
     Q[l] [B*R,64,576] bf16, KV[l] [P,64,576] e4m3 + KV_scale[l] [P,64] fp32,
     block_table [B,max_pages] int32, seq_lens [B] int32.
@@ -212,6 +230,14 @@ def make_decode(spec: DecodeSpec, device=None, ctx=None, layers=None) -> dict:
     q = _normal(sub_seed(s, 0, T_QIDX), B * IDX_HEADS * IDX_DIM, device)
     out["q_idx"] = _bf16(q, device).reshape(B, IDX_HEADS, IDX_DIM)
     out["w"] = _f32(_normal(sub_seed(s, 0, T_W), B * IDX_HEADS, device), device).reshape(B, IDX_HEADS)
+    out["topk_per_row"] = bool(spec.topk_per_row)
+    if spec.topk_per_row and R > 1:
+        if spec.n_layers > 4:
+            raise ValueError("per-row Top-k inputs are drawn for one IndexShare group only")
+        qd = _bf16(_normal(sub_seed(s, 0, T_QIDX_DRAFT), B * (R - 1) * IDX_HEADS * IDX_DIM, device), device)
+        wd = _f32(_normal(sub_seed(s, 0, T_W_DRAFT), B * (R - 1) * IDX_HEADS, device), device)
+        out["q_idx"] = _cat_rows(out["q_idx"], qd.reshape(B, R - 1, IDX_HEADS, IDX_DIM), (B * R, IDX_HEADS, IDX_DIM))
+        out["w"] = _cat_rows(out["w"], wd.reshape(B, R - 1, IDX_HEADS), (B * R, IDX_HEADS))
     out["idx_keys"], out["idx_key_scale"] = _fp8_pool(sub_seed(s, 0, T_KIDX), total, IDX_DIM, device)
     layers = range(spec.n_layers) if layers is None else layers
     out["Q"], out["KV"], out["KV_scale"] = [], [], []

@@ -33,9 +33,22 @@ def test_decode_counts():
     assert c["mla_bytes_per_layer"] == sel * 580.0 + 15 * 64 * (576 + 512) * 2.0
 
 
+def test_decode_per_row_topk_counts():
+    # every row scores the same keys with its own query and gathers its own selection
+    ctx = np.array([1000, 5000, 70000])
+    reuse = bench.algorithmic_counts(WORKLOADS["decode_b32_mtp4"], ctx)
+    c = bench.algorithmic_counts(WORKLOADS["decode_b32_mtp4_verify"], ctx)
+    sel = 1000 + 2048 + 2048
+    assert c["tokens"] == reuse["tokens"] == 15
+    assert c["indexer_flops"] == 5 * reuse["indexer_flops"] == 5 * 8192.0 * ctx.sum()
+    assert c["indexer_bytes"] == reuse["indexer_bytes"]          # the keys are needed once
+    assert c["mla_flops_per_layer"] == reuse["mla_flops_per_layer"]
+    assert c["mla_bytes_per_layer"] == 5 * sel * 580.0 + 15 * 64 * (576 + 512) * 2.0
+
+
 def test_workload_configs_name_every_bench_workload():
     for name in ["tiny_prefill", "prefill_32k", "prefill_128k_fp8", "decode_b32_mtp4", "decode_b32_d0",
-                 "decode_1m_mtp5"]:
+                 "decode_b32_mtp4_verify", "decode_1m_mtp5"]:
         spec, cfg = bench.workload_config(name)
         assert cfg["workload"] == name
     spec, cfg = bench.workload_config("decode_b32_d0")

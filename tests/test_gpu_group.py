@@ -1,7 +1,8 @@
 """IndexShare group (Full layer + Shared layers) through the C ABI against the fp64 oracle.
 
 Covers the 512-token tiny prefill workload in full, a scaled FP8-indexer prefill, a
-scaled batched decode with MTP rows and paged FP8 caches, and the reuse-handle rules.
+scaled batched decode with MTP rows and paged FP8 caches (rows reusing row 0's Top-k, and
+rows taking their own), and the reuse-handle rules.
 Tolerances as in test_gpu_kernels.py; the FP8 indexer path also checks end-to-end
 relative L2 <= 3e-2 against the oracle run on unquantised bf16 inputs.
 """
@@ -141,6 +142,47 @@ def test_decode_group_mtp_paged():
                 ref, _ = O.sparse_mla_row(O.bf16_to_f64(inp["Q"][l][row]), kv, idx[b], inp["softmax_scale"])
                 ma, rel = attn_errors(outs[l][row], ref)
                 assert ma <= 2e-2 and rel <= 5e-3, (l, row, ma, rel)
+
+
+def test_decode_verification_rows_take_their_own_topk():
+    """Per-row Top-k for MTP verification rows: each of the R rows of a sequence is its own entry of
+    a paged view over the sequence's pages, scored with its own indexer query; every row's set and
+    its attention in both layers match the fp64 oracle of that policy."""
+    spec = DecodeSpec("v", batch=4, ctx_lo=500, ctx_hi=12000, rows_per_seq=3, k=256, n_layers=2, seed=10,
+                      topk_per_row=True)
+    inp = make_decode(spec)
+    R, ctx, bt = spec.rows_per_seq, inp["ctx"], inp["block_table"]
+    ctx_d, bt_d = i32_dev(ctx), i32_dev(bt)
+    keys = dsa.paged_view(u8_dev(inp["idx_keys"]), f32_dev(inp["idx_key_scale"]), bt_d, ctx_d, rows_per_seq=R)
+    kvs = [dsa.paged_view(u8_dev(inp["KV"][l]), f32_dev(inp["KV_scale"][l]), bt_d, ctx_d, rows_per_seq=R)
+           for l in range(2)]
+    g = dsa.IndexShareGroup(bf16_dev(inp["q_idx"]), f32_dev(inp["w"]), keys, spec.k,
+                            [bf16_dev(x) for x in inp["Q"]], kvs, inp["softmax_scale"],
+                            indexer_dtype=dsa.DSA_E4M3, q_rows_per_idx_row=1)
+    out, lse = g.forward()
+    dsa.sync_status()
+    idx = g.idx.cpu().numpy()
+    assert idx.shape == (spec.batch * R, spec.k)
+    q8, sq = O.quantize_e4m3_rows(inp["q_idx"], 128)
+    qv = O.e4m3_to_f64(q8) * sq.reshape(-1, 32, 1)
+    outs = [O.bf16_to_f64(bf16_host(o)) for o in out]
+    lses = [x.cpu().numpy() for x in lse]
+    for b in range(spec.batch):
+        n = int(ctx[b])
+        kk = O.paged_rows(inp["idx_keys"], inp["idx_key_scale"], bt[b], n)
+        kv = [O.paged_rows(inp["KV"][l], inp["KV_scale"][l], bt[b], n) for l in range(2)]
+        for r in range(R):
+            row = b * R + r
+            sc = O.indexer_scores(qv[row:row + 1], inp["w"][row:row + 1], kk, [n])[0]
+            check_topk_sets(idx[row], sc, n, spec.k)
+            for l in range(2):
+                ref, ref_lse = O.sparse_mla_row(O.bf16_to_f64(inp["Q"][l][row]), kv[l], idx[row],
+                                                inp["softmax_scale"])
+                ma, rel = attn_errors(outs[l][row], ref)
+                assert ma <= 2e-2 and rel <= 5e-3, (l, row, ma, rel)
+                assert np.max(np.abs(lses[l][row] - ref_lse)) <= 2e-3, (l, row)
+    # the draft rows' own queries select other sets than row 0's
+    assert any(set(idx[b * R + 1]) != set(idx[b * R]) for b in range(spec.batch))
 
 
 def test_decode_group_replays_from_a_captured_cuda_graph():

@@ -222,6 +222,52 @@ def test_decode_mtp_rows_share_row0_indices():
         assert (g["idx"][b] < n).all()
 
 
+def _per_row_decode_inputs():
+    spec = DecodeSpec("t", batch=2, ctx_lo=70, ctx_hi=260, rows_per_seq=3, k=16, n_layers=2, seed=3,
+                      topk_per_row=True)
+    return make_decode(spec)
+
+
+def _reuse_inputs_with_query_row(inp, r):
+    """The same decode step under the reuse policy, with draft row r's indexer query and weights
+    standing as each sequence's own."""
+    R = inp["rows_per_seq"]
+    return dict(inp, q_idx=inp["q_idx"][r::R], w=inp["w"][r::R], topk_per_row=False)
+
+
+def test_per_row_topk_with_equal_row_queries_is_the_reuse_policy(fn=None):
+    """V1 reduces to R7 when all rows of a sequence carry row 0's indexer query and weights."""
+    fn = fn or O.group_decode_per_row
+    inp = _per_row_decode_inputs()
+    R = inp["rows_per_seq"]
+    same = dict(inp, q_idx=np.repeat(inp["q_idx"][::R], R, axis=0), w=np.repeat(inp["w"][::R], R, axis=0))
+    g, ref = fn(same), O.group_decode(_reuse_inputs_with_query_row(inp, 0))
+    for b in range(2):
+        for r in range(R):
+            assert np.array_equal(g["idx"][b * R + r], ref["idx"][b])
+            for l in range(2):
+                assert np.array_equal(g["O"][l][b * R + r], ref["O"][l][b * R + r])
+                assert g["lse"][l][b * R + r] == pytest.approx(ref["lse"][l][b * R + r], abs=0, rel=0)
+
+
+def test_per_row_topk_row_r_is_the_reuse_policy_with_row_r_query(fn=None):
+    """Row b*R + r of V1 equals row b*R + r of R7 run with row r's indexer query: each row keeps
+    the selection of its own query, over its own sequence's keys."""
+    fn = fn or O.group_decode_per_row
+    inp = _per_row_decode_inputs()
+    R = inp["rows_per_seq"]
+    g = fn(inp)
+    differ = 0
+    for r in range(R):
+        ref = O.group_decode(_reuse_inputs_with_query_row(inp, r))
+        for b in range(2):
+            assert np.array_equal(g["idx"][b * R + r], ref["idx"][b])
+            differ += not np.array_equal(g["idx"][b * R + r], g["idx"][b * R])
+            for l in range(2):
+                assert np.array_equal(g["O"][l][b * R + r], ref["O"][l][b * R + r])
+    assert differ > 0      # the draft rows' own queries select other sets than row 0's
+
+
 def test_paged_rows_follow_block_table():
     spec = DecodeSpec("t", batch=3, ctx_lo=65, ctx_hi=300, rows_per_seq=1, k=8, n_layers=1, seed=2)
     inp = make_decode(spec)
@@ -292,3 +338,14 @@ def test_planted_attention_mistakes_are_caught(old, new):
     bad = _mutant(O.sparse_mla_row, old, new)
     with pytest.raises(AssertionError):
         test_sparse_equals_dense_when_k_covers_history(bad)
+
+
+@pytest.mark.parametrize("old,new", [
+    ("qv[row:row + 1], w[row:row + 1]", "qv[b * R:b * R + 1], w[b * R:b * R + 1]"),   # row 0's query for all
+    ("kvrows, idx[row]", "kvrows, idx[b * R]"),                                        # row 0's selection
+    ('paged_rows(inp["KV"][l]', 'paged_rows(inp["KV"][0]'),                             # layer 0's cache
+])
+def test_planted_per_row_policy_mistakes_are_caught(old, new):
+    bad = _mutant(O.group_decode_per_row, old, new)
+    with pytest.raises(AssertionError):
+        test_per_row_topk_row_r_is_the_reuse_policy_with_row_r_query(bad)

@@ -49,3 +49,23 @@ def test_prefill_shapes():
     inp = make_prefill(PrefillSpec("x", L=40, k=8), layers=[0, 1])
     assert inp["q_idx"].shape == (40, 32, 128) and inp["Q"][1].shape == (40, 64, 576)
     assert inp["KV"][0].dtype == np.uint16 and inp["w"].dtype == np.float32
+
+
+def test_per_row_topk_recipe_keeps_row0_of_the_reuse_recipe():
+    import dataclasses
+    from synth import make_decode
+    spec = WORKLOADS["decode_b32_mtp4_verify"]
+    assert spec.topk_per_row and spec.rows_per_seq == 5
+    small = dataclasses.replace(spec, batch=3, ctx_lo=100, ctx_hi=400, k=32, n_layers=1)
+    reuse = make_decode(dataclasses.replace(small, topk_per_row=False))
+    per_row = make_decode(small)
+    R = small.rows_per_seq
+    assert per_row["q_idx"].shape == (3 * R, 32, 128) and per_row["w"].shape == (3 * R, 32)
+    assert np.array_equal(per_row["q_idx"][::R], reuse["q_idx"]) and np.array_equal(per_row["w"][::R], reuse["w"])
+    assert not np.array_equal(per_row["q_idx"][1::R], reuse["q_idx"])
+    for key in ("ctx", "block_table", "idx_keys", "idx_key_scale"):
+        assert np.array_equal(per_row[key], reuse[key])
+    assert np.array_equal(per_row["Q"][0], reuse["Q"][0]) and np.array_equal(per_row["KV"][0], reuse["KV"][0])
+    on_torch = make_decode(small, device="cpu")
+    assert np.array_equal(on_torch["q_idx"].view(torch.int16).numpy(), per_row["q_idx"].view(np.int16))
+    assert np.array_equal(on_torch["w"].numpy(), per_row["w"])
