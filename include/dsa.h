@@ -112,6 +112,24 @@ dsa_status dsa_quant_e4m3(const void* x_bf16, int64_t n_vec, int32_t vec_len, ui
                           void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Step a1 on the decode side: append new tokens to a paged FP8 cache (same pages and format
+ * as the paged dsa_cache_view: e4m3 codes [n_pages, 64, dim] + fp32 scales [n_pages, 64], one
+ * scale per token, rule as in dsa_quant_e4m3 over the token's whole row).
+ *   x_bf16      [n_rows, dim] bf16, dim 128 (indexer keys) or 576 (latent rows); 16-byte aligned
+ *   seq         [n_rows] int32 sequence of each row, or NULL for row r -> sequence r
+ *   pos         [n_rows] int32 position of each row in its sequence
+ *   block_table [batch, max_pages] int32: slot of (b, t) = page block_table[b][t / 64], entry t % 64
+ *   pool        [n_pages, 64, dim] uint8 (16-byte aligned), pool_scale [n_pages, 64] fp32: written
+ *               at the rows' slots only
+ * Each (sequence, position) may appear at most once per call.  Host-side errors: null or
+ * misaligned pointers, dim not 128 / 576, negative sizes.  A row whose sequence, position or page
+ * is out of range is skipped on the device and reported as DSA_ERR_BOUNDS by dsa_sync_status.
+ */
+dsa_status dsa_cache_write_e4m3(const void* x_bf16, int32_t n_rows, int32_t dim, const int32_t* seq,
+                                const int32_t* pos, const int32_t* block_table, int32_t batch, int32_t max_pages,
+                                int32_t n_pages, uint8_t* pool, float* pool_scale, void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * Steps a2+a3: lightweight-indexer scores (forum.sourcefind.cn "IndexShare：省掉3/4的索引计算";
  * 32 heads, ailearn architecture card), with the ReLU, per-head weight and causal mask
  * fused into the tensor-core epilogue:

@@ -25,7 +25,7 @@ EXPORTS = [
     "dsa_sparse_mla_workspace_bytes", "dsa_sparse_mla_attn", "dsa_group_workspace_bytes",
     "indexshare_group_forward", "dsa_layer_is_full", "dsa_layer_producer", "dsa_status_str",
     "dsa_last_error", "dsa_abi_version", "dsa_abi_sizeof", "dsa_sync_status", "dsa_debug_bounded_wait",
-    "dsa_set_wait_limit_ns", "dsa_launch_count", "dsa_topk_no_alloc",
+    "dsa_set_wait_limit_ns", "dsa_launch_count", "dsa_topk_no_alloc", "dsa_cache_write_e4m3",
 ]
 
 
@@ -68,6 +68,8 @@ def load(path: str = LIB_PATH):
     S = c_int32
     sig = {
         "dsa_quant_e4m3": (S, [c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p]),
+        "dsa_cache_write_e4m3": (S, [c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_int32, c_int32,
+                                     c_int32, c_void_p, c_void_p, c_void_p]),
         "dsa_indexer_score": (S, [c_void_p, c_int32, c_void_p, c_void_p, c_int32, c_int32, POINTER(CacheView),
                                   c_void_p, c_int64, c_void_p]),
         "dsa_topk_workspace_bytes": (c_size_t, [c_int32, c_int64, c_int32]),
@@ -156,6 +158,17 @@ def quant_e4m3(x, codes=None, scale=None):
     scale = torch.empty(n_vec, dtype=torch.float32, device=x.device) if scale is None else scale
     _check(load().dsa_quant_e4m3(x.data_ptr(), n_vec, 128, codes.data_ptr(), scale.data_ptr(), _stream()))
     return codes, scale
+
+
+def cache_write_e4m3(x, pos, block_table, pool, pool_scale, seq=None):
+    """a1 for decode: rows x [n,dim] bf16 (dim 128 or 576) quantised per token into their slots of
+    the paged pool [n_pages,64,dim] uint8 / pool_scale [n_pages,64] fp32; row r goes to sequence
+    seq[r] (r when seq is None) at position pos[r] through block_table [B,max_pages] int32."""
+    n, dim = x.shape
+    _check(load().dsa_cache_write_e4m3(x.data_ptr(), n, dim, _ptr(seq), pos.data_ptr(), block_table.data_ptr(),
+                                       block_table.shape[0], block_table.shape[1], pool.shape[0], pool.data_ptr(),
+                                       pool_scale.data_ptr(), _stream()))
+    return pool, pool_scale
 
 
 def indexer_score(q, w, keys: CacheView, scores, q_scale=None, q_pos0: int = 0):

@@ -629,6 +629,25 @@ dsa_status dsa_quant_e4m3(const void* x_bf16, int64_t n_vec, int32_t vec_len, ui
   return cuda_check(cudaGetLastError(), "quant launch");
 }
 
+dsa_status dsa_cache_write_e4m3(const void* x_bf16, int32_t n_rows, int32_t dim, const int32_t* seq,
+                                const int32_t* pos, const int32_t* block_table, int32_t batch, int32_t max_pages,
+                                int32_t n_pages, uint8_t* pool, float* pool_scale, void* stream) {
+  if (dim != 128 && dim != 576) return fail(DSA_ERR_UNSUPPORTED, "cache write dim %d (128 or 576)", dim);
+  if (n_rows < 0 || batch < 0 || max_pages < 0 || n_pages < 0) return fail(DSA_ERR_INVALID_ARG, "negative size");
+  if (n_rows == 0) return DSA_OK;
+  if (!x_bf16 || !aligned16(x_bf16) || !pos || !block_table || !pool || !aligned16(pool) || !pool_scale)
+    return fail(DSA_ERR_INVALID_ARG, "null or misaligned pointer");
+  if (batch == 0 || max_pages == 0 || n_pages == 0) return fail(DSA_ERR_INVALID_ARG, "empty cache");
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  const int64_t blocks = (static_cast<int64_t>(n_rows) + 7) / 8;
+  cache_write_e4m3_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(x_bf16), n_rows, dim, seq, pos, block_table, batch, max_pages, n_pages, pool,
+      pool_scale, ds->status);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "cache write launch");
+}
+
 dsa_status dsa_indexer_score(const void* q, int32_t q_dtype, const float* q_scale, const float* w, int32_t n_q,
                              int32_t q_pos0, const dsa_cache_view* keys, float* scores, int64_t ld_scores,
                              void* stream) {

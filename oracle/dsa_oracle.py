@@ -55,7 +55,7 @@ import math
 import numpy as np
 
 __all__ = [
-    "bf16_to_f64", "e4m3_to_f64", "quantize_e4m3_rows", "indexer_scores", "topk_rows",
+    "bf16_to_f64", "e4m3_to_f64", "quantize_e4m3_rows", "cache_write_e4m3", "indexer_scores", "topk_rows",
     "topk_row", "sparse_mla_row", "dense_causal_attention_row", "sparse_mla",
     "group_prefill", "group_decode", "group_decode_per_row", "layer_schedule", "indexer_param_count",
     "E4M3_MAX", "IDX_HEADS", "IDX_DIM", "MLA_HEADS", "D_QK", "D_V", "PAGE",
@@ -128,6 +128,20 @@ def quantize_e4m3_rows(x_bf16_bits, vec_len: int):
     v = (x / scale[:, None]).astype(np.float32)          # IEEE fp32 division
     codes = _encode_e4m3_rne_sat(v).reshape(np.asarray(x_bf16_bits).shape)
     return codes, scale
+
+
+def cache_write_e4m3(pool, scale, block_table, x_bf16_bits, seq, pos):
+    """Decode-side FP8 cache write (R5, R10): new row r is quantised with one scale over its whole
+    row and stored at entry pos[r] % 64 of page block_table[seq[r]][pos[r] // 64].  Returns
+    written copies of pool [n_pages,64,dim] and scale [n_pages,64]."""
+    pool, scale = np.array(pool, copy=True), np.array(scale, copy=True)
+    codes, sc = quantize_e4m3_rows(x_bf16_bits, pool.shape[2])
+    for r in range(len(pos)):
+        b, t = int(seq[r]), int(pos[r])
+        page = int(block_table[b][t // PAGE])
+        pool[page, t % PAGE] = codes[r]
+        scale[page, t % PAGE] = sc[r]
+    return pool, scale
 
 
 # ----------------------------------------------------------------------------- indexer

@@ -95,6 +95,42 @@ def test_quant_e4m3_bit_exact():
     assert np.array_equal(codes.cpu().numpy(), rc)
 
 
+def test_cache_write_e4m3_bit_exact():
+    """Decode-side a1: new rows quantised into their paged slots, bit-exact with the oracle for
+    index keys (128) and latent rows (576), other slots untouched; a row whose page is not in the
+    block table is skipped and reported."""
+    spec = DecodeSpec("c", batch=3, ctx_lo=100, ctx_hi=700, rows_per_seq=1, k=8, n_layers=1, seed=12)
+    inp = make_decode(spec)
+    bt, ctx = inp["block_table"], inp["ctx"]
+    rng = np.random.default_rng(3)
+    for dim, pool, scale in ((128, inp["idx_keys"], inp["idx_key_scale"]), (576, inp["KV"][0], inp["KV_scale"][0])):
+        pairs = sorted({(int(b), int(t)) for b, t in zip(rng.integers(0, 3, 80), rng.integers(0, 100, 80))})[:40]
+        seq = np.array([q[0] for q in pairs], dtype=np.int32)
+        pos = np.array([q[1] for q in pairs], dtype=np.int32)
+        x = normal_np(20 + dim, 0, len(pairs) * dim).reshape(-1, dim) * 3.0
+        x[5] = 0.0                      # all-zero row: scale 1
+        x[7, 3] = 2e4                   # one large element: the rest of its row rounds to small codes
+        bits = bf16_bits_np(x)
+        ref_pool, ref_scale = O.cache_write_e4m3(pool, scale, bt, bits, seq, pos)
+        pool_d, scale_d = u8_dev(pool), f32_dev(scale)
+        dsa.cache_write_e4m3(bf16_dev(bits), i32_dev(pos), i32_dev(bt), pool_d, scale_d, seq=i32_dev(seq))
+        dsa.sync_status()
+        assert np.array_equal(pool_d.cpu().numpy(), ref_pool)
+        assert np.array_equal(scale_d.cpu().numpy(), ref_scale)
+    # sequence 0 at a position past its pages (block-table entry -1): skipped and reported
+    t_out = int((ctx[0] + 63) // 64) * 64   # first logical page past the sequence (or past max_pages)
+    seq = np.array([0, 1], dtype=np.int32)
+    pos = np.array([t_out, 5], dtype=np.int32)
+    bits = bf16_bits_np(normal_np(40, 0, 2 * 128).reshape(2, 128))
+    pool_d, scale_d = u8_dev(inp["idx_keys"]), f32_dev(inp["idx_key_scale"])
+    dsa.cache_write_e4m3(bf16_dev(bits), i32_dev(pos), i32_dev(bt), pool_d, scale_d, seq=i32_dev(seq))
+    with pytest.raises(dsa.DsaError) as err:
+        dsa.sync_status()
+    assert err.value.status == dsa.binding.DSA_ERR_BOUNDS
+    ref_pool, ref_scale = O.cache_write_e4m3(inp["idx_keys"], inp["idx_key_scale"], bt, bits[1:], seq[1:], pos[1:])
+    assert np.array_equal(pool_d.cpu().numpy(), ref_pool) and np.array_equal(scale_d.cpu().numpy(), ref_scale)
+
+
 # ----------------------------------------------------------------------------- a4
 
 

@@ -279,6 +279,26 @@ def test_paged_rows_follow_block_table():
     assert np.array_equal(rows[129], O.e4m3_to_f64(inp["KV"][0][p, s]) * float(inp["KV_scale"][0][p, s]))
 
 
+def test_cache_write_fills_the_slots_paged_rows_reads(fn=None):
+    """Writing every position of a sequence, in any order, makes its paged rows read back as the
+    dequantised per-token quantisation of the written rows; other sequences' slots are untouched."""
+    fn = fn or O.cache_write_e4m3
+    spec = DecodeSpec("t", batch=3, ctx_lo=65, ctx_hi=300, rows_per_seq=1, k=8, n_layers=1, seed=6)
+    inp = make_decode(spec)
+    bt, ctx = inp["block_table"], inp["ctx"]
+    for dim, pool, scale in ((128, inp["idx_keys"], inp["idx_key_scale"]), (576, inp["KV"][0], inp["KV_scale"][0])):
+        n = int(ctx[1])
+        x = np.asarray(make_prefill(PrefillSpec("x", L=n, k=8), layers=[0])["KV"][0][:, :dim])
+        order = np.random.default_rng(dim).permutation(n)
+        new_pool, new_scale = fn(pool, scale, bt, x[order], np.full(n, 1), order)
+        codes, sc = O.quantize_e4m3_rows(x, dim)
+        assert np.array_equal(O.paged_rows(new_pool, new_scale, bt[1], n),
+                              O.e4m3_to_f64(codes) * sc.astype(np.float64)[:, None])
+        for b in (0, 2):
+            m = int(ctx[b])
+            assert np.array_equal(O.paged_rows(new_pool, new_scale, bt[b], m), O.paged_rows(pool, scale, bt[b], m))
+
+
 def test_schedule_matches_pages():
     sch = O.layer_schedule(GOLD["n_layers"]["value"])
     full = [l for l, f, _ in sch if f]
@@ -349,3 +369,14 @@ def test_planted_per_row_policy_mistakes_are_caught(old, new):
     bad = _mutant(O.group_decode_per_row, old, new)
     with pytest.raises(AssertionError):
         test_per_row_topk_row_r_is_the_reuse_policy_with_row_r_query(bad)
+
+
+@pytest.mark.parametrize("old,new", [
+    ("t % PAGE] = codes[r]", "(t + 1) % PAGE] = codes[r]"),             # slot off by one
+    ("block_table[b][t // PAGE]", "block_table[0][t // PAGE]"),          # first sequence's pages
+    ("scale[page, t % PAGE] = sc[r]", "scale[page, t % PAGE] = 1.0"),    # scale not stored
+])
+def test_planted_cache_write_mistakes_are_caught(old, new):
+    bad = _mutant(O.cache_write_e4m3, old, new)
+    with pytest.raises(AssertionError):
+        test_cache_write_fills_the_slots_paged_rows_reads(bad)
