@@ -91,6 +91,35 @@ def test_host_validation_rejects_before_launch(lib):
         == B.DSA_ERR_INVALID_ARG
 
 
+def test_cache_write_validation(lib):
+    args = dict(seq=None, pos=32, bt=48, batch=2, max_pages=4, n_pages=8, pool=64, scale=80)
+
+    def call(x=16, n=4, dim=128, **kw):
+        a = dict(args, **kw)
+        return lib.dsa_cache_write_e4m3(x, n, dim, a["seq"], a["pos"], a["bt"], a["batch"], a["max_pages"],
+                                        a["n_pages"], a["pool"], a["scale"], None)
+    assert call(dim=512) == B.DSA_ERR_UNSUPPORTED           # neither an index key nor a latent row
+    assert call(n=-1) == B.DSA_ERR_INVALID_ARG
+    assert call(x=17) == B.DSA_ERR_INVALID_ARG and "aligned" in _err(lib)
+    assert call(pool=65) == B.DSA_ERR_INVALID_ARG
+    assert call(pos=None) == B.DSA_ERR_INVALID_ARG
+    assert call(n_pages=0) == B.DSA_ERR_INVALID_ARG and "empty" in _err(lib)
+    assert call(n=0) == B.DSA_OK                            # nothing to write: no launch
+
+
+def test_per_row_paged_view_repeats_tables_not_pages():
+    import torch
+    pool = torch.zeros(6, 64, 128, dtype=torch.uint8)
+    scale = torch.ones(6, 64)
+    bt = torch.tensor([[4, 1, -1], [0, 5, 2]], dtype=torch.int32)
+    lens = torch.tensor([100, 150], dtype=torch.int32)
+    v = dsa.paged_view(pool, scale, bt, lens, rows_per_seq=3)
+    assert v.batch == 6 and v.max_pages == 3 and v.data == pool.data_ptr() and v.n_tokens == 6 * 64
+    assert v._keep[2].tolist() == [[4, 1, -1]] * 3 + [[0, 5, 2]] * 3
+    assert v._keep[3].tolist() == [100] * 3 + [150] * 3
+    assert v.block_table == v._keep[2].data_ptr() and v.seq_lens == v._keep[3].data_ptr()
+
+
 def test_group_handle_checks(lib):
     a = B.GroupArgs()
     a.q_idx, a.w = 16, 32
