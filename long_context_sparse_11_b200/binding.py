@@ -244,9 +244,8 @@ class IndexShareGroup:
         for i, (qq, vv) in enumerate(zip(q, kv)):
             a.q[i], a.kv[i], a.out[i], a.lse[i] = qq.data_ptr(), vv, self.out[i].data_ptr(), self.lse[i].data_ptr()
         lib = load()
+        # 0 when the arguments are invalid: forward() then returns the validation error itself
         need = lib.dsa_group_workspace_bytes(ctypes.byref(a))
-        if need == 0 and lib.dsa_last_error():
-            pass
         self.workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
         a.workspace, a.workspace_bytes = self.workspace.data_ptr(), self.workspace.numel()
         self.args = a
