@@ -23,8 +23,8 @@ namespace idx {
 constexpr int BLOCK_KEYS = 128;
 constexpr int UNIT_TILES = 32;  // key tiles per work unit (default; decode may use fewer)
 
-// ReLU split between two pipes.  max(x, 0) runs on the ALU pipe, which the epilogue saturates
-// first; for P of the 16 head pairs the epilogue instead forms x + |x| = 2 max(x, 0) with one
+// ReLU split between two pipes.  max(x, 0) runs on the ALU pipe, the epilogue's busiest; for P
+// of the 16 head pairs the epilogue instead forms x + |x| = 2 max(x, 0) with one
 // add on the FMA pipe and the staged weight of those heads is halved, so w * max(x, 0) is
 // reproduced exactly (0.5 w * 2x = w * x for every finite accumulator x).  The P pairs are
 // spread evenly over the 16.
