@@ -3,7 +3,8 @@
 Closed forms: a causal prefill of L rows has L(L+1)/2 indexer pairs of 8,192 flops
 (32 heads x 128 dims x 2) and sum_t min(k, t+1) selected keys of 139,264 attention flops
 (64 heads x (576 + 512) x 2); a decode sequence of context N reads 132 B per key in the
-indexer (128-byte e4m3 code + 4-byte scale) and gathers 580 B per selected key.
+indexer (128-byte e4m3 code + 4-byte scale) and gathers 580 B per selected key.  The reference
+arm's JSON line is checked end to end on the smallest workload.
 """
 import numpy as np
 
@@ -59,3 +60,27 @@ def test_mla_dram_bytes_per_row_is_queries_plus_outputs():
     # the ncu-derived traffic per query row sits just above the queries in and outputs out
     q_out = 64 * 576 * 2 + 64 * 512 * 2
     assert q_out <= bench.MLA_DRAM_BYTES_PER_ROW_BF16 <= 1.1 * q_out
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints exactly one JSON line
+    with the contract keys; it runs here on the CPU on the smallest workload."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload",
+                          "tiny_prefill", "--steps", "1", "--warmup", "0", "--ref-seconds", "1"],
+                         capture_output=True, text=True, timeout=300, cwd=root)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert d["config"]["workload"] == "tiny_prefill"
