@@ -120,6 +120,21 @@ def test_per_row_paged_view_repeats_tables_not_pages():
     assert v.block_table == v._keep[2].data_ptr() and v.seq_lens == v._keep[3].data_ptr()
 
 
+def test_empty_inputs_are_a_no_op(lib):
+    """Zero rows (an empty batch, a chunk with no queries) succeed with no launch and no device
+    access, whatever the data pointers are."""
+    before = lib.dsa_launch_count()
+    assert lib.dsa_quant_e4m3(None, 0, 128, None, None, None) == B.DSA_OK
+    v = B.CacheView(16, None, None, None, 128, 100, 128, B.DSA_BF16, 0, 0)
+    assert lib.dsa_indexer_score(None, B.DSA_BF16, None, None, 0, 0, ctypes.byref(v), None, 128, None) == B.DSA_OK
+    assert lib.dsa_topk(None, 64, 0, None, 1, 64, 8, None, None, 0, None) == B.DSA_OK
+    assert lib.dsa_topk_no_alloc(None, 64, 0, None, 1, 64, 8, None, None) == B.DSA_OK
+    v = B.CacheView(16, None, None, None, 576, 100, 576, B.DSA_BF16, 0, 0)
+    assert lib.dsa_sparse_mla_attn(None, ctypes.byref(v), None, 0, 1, 8, 0.04, None, None, None, 0, None) == B.DSA_OK
+    assert lib.dsa_cache_write_e4m3(None, 0, 576, None, None, None, 1, 1, 1, None, None, None) == B.DSA_OK
+    assert lib.dsa_launch_count() == before
+
+
 def test_group_handle_checks(lib):
     a = B.GroupArgs()
     a.q_idx, a.w = 16, 32
