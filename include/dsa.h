@@ -112,9 +112,12 @@ dsa_status dsa_quant_e4m3(const void* x_bf16, int64_t n_vec, int32_t vec_len, ui
                           void* stream);
 
 /* ---------------------------------------------------------------------------------------
- * Step a1 on the decode side: append new tokens to a paged FP8 cache (same pages and format
- * as the paged dsa_cache_view: e4m3 codes [n_pages, 64, dim] + fp32 scales [n_pages, 64], one
- * scale per token, rule as in dsa_quant_e4m3 over the token's whole row).
+ * Step a1 on the decode side: append new tokens to a paged FP8 cache (the FP8 KV cache of the
+ * pages cited at dsa_quant_e4m3; the 64-token page is this library's choice, as for the paged
+ * dsa_cache_view, since the pages give no block size).  Same pages and format as that view:
+ * e4m3 codes [n_pages, 64, dim] + fp32 scales [n_pages, 64], one scale per token, rule as in
+ * dsa_quant_e4m3 over the token's whole row.  Ownership: the caller owns every buffer; the call
+ * writes only the rows' slots of pool and pool_scale, asynchronously on the stream.
  *   x_bf16      [n_rows, dim] bf16, dim 128 (indexer keys) or 576 (latent rows); 16-byte aligned
  *   seq         [n_rows] int32 sequence of each row, or NULL for row r -> sequence r
  *   pos         [n_rows] int32 position of each row in its sequence
