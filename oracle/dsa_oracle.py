@@ -47,6 +47,10 @@ V1  MTP verification, the alternative to R7: each of the 1+d query rows of a seq
     is what that reuse saves, so it is built to be compared against it.
 R8  78-layer schedule: Full at 0-based layers 0, 1 and 2 + 4g; the rest Shared, each
     reusing the preceding Full layer ([ailearn] "IndexShare：四层共用一次搜索结果").
+R10 The paged FP8 latent cache holds all 576 dims as e4m3 with one fp32 scale per token
+    (the pages name an FP8 KV cache, [forum] "vLLM推理启动", but not its layout).
+R11 Paged caches: token s of sequence b sits in page block_table[b][s // 64], slot s % 64
+    (the pages give no block size).
 """
 from __future__ import annotations
 
@@ -131,7 +135,7 @@ def quantize_e4m3_rows(x_bf16_bits, vec_len: int):
 
 
 def cache_write_e4m3(pool, scale, block_table, x_bf16_bits, seq, pos):
-    """Decode-side FP8 cache write (R5, R10): new row r is quantised with one scale over its whole
+    """Decode-side FP8 cache write (R5, R10, R11): new row r is quantised with one scale over its whole
     row and stored at entry pos[r] % 64 of page block_table[seq[r]][pos[r] // 64].  Returns
     written copies of pool [n_pages,64,dim] and scale [n_pages,64]."""
     pool, scale = np.array(pool, copy=True), np.array(scale, copy=True)
@@ -275,7 +279,7 @@ def group_prefill(inp: dict, rows, fp8_indexer: bool = False, idx_override=None)
 
 
 def paged_rows(pool, scale, block_table_row, n: int) -> np.ndarray:
-    """Dequantised cache rows 0..n-1 of one sequence: row s lives in page bt[s // 64], slot s % 64."""
+    """Dequantised cache rows 0..n-1 of one sequence (R10, R11): row s lives in page bt[s // 64], slot s % 64."""
     s = np.arange(n)
     pages = np.asarray(block_table_row)[s // PAGE]
     slots = s % PAGE
