@@ -21,12 +21,14 @@
 // sub-tiles (one 128-dim block of V) its own "empty" barrier, committed when the PV MMAs of
 // that block complete.  The gather of tile j+1 therefore streams into the sub-tiles that
 // PV(j) has finished with while PV(j) still runs on the others, and S^T(j+1) starts as soon
-// as its first sub-tile lands.  CTAs are persistent over (query row, key split) items.
+// as its first sub-tile lands.  CTAs are persistent over (query row, key split) items, or,
+// for short decode batches, over equal stream-K ranges of the (row, key tile) sequence whose
+// cut rows are merged by the combine kernel.
 //
 // Rows are gathered with 16-byte cp.async whose completion the hardware reports to the
-// sub-tile's barrier (bf16 cache), or 16-byte loads + e4m3 -> f16 conversion (paged FP8 cache; the MMAs then run
-// kind::f16 on f16 operands, exact for e4m3 values; the per-token scale is applied to the
-// logits and folded into P^T).
+// sub-tile's barrier (bf16 cache), or with 16-byte loads + e4m3 -> f16 conversion (paged FP8
+// cache; the MMAs then run kind::f16 on f16 operands, exact for e4m3 values; the per-token
+// scale is applied to the logits and folded into P^T).
 //
 // Warps 0..SM_WARPS-1: softmax / output (warp w: lane quadrant w%4, HPW heads from HPW*(w/4)),
 // and on the FP8 path part of the gather; the next GA_WARPS (7) warps: query rows and the KV gather; the
