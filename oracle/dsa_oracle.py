@@ -59,9 +59,9 @@ import math
 import numpy as np
 
 __all__ = [
-    "bf16_to_f64", "e4m3_to_f64", "quantize_e4m3_rows", "cache_write_e4m3", "indexer_scores", "topk_rows",
-    "topk_row", "sparse_mla_row", "dense_causal_attention_row", "sparse_mla",
-    "group_prefill", "group_decode", "group_decode_per_row", "layer_schedule", "indexer_param_count",
+    "bf16_to_f64", "e4m3_to_f64", "quantize_e4m3_rows", "cache_write_e4m3", "indexer_scores",
+    "topk_row", "sparse_mla_row", "dense_causal_attention_row", "prefill_tables",
+    "group_prefill", "paged_rows", "group_decode", "group_decode_per_row", "layer_schedule", "indexer_param_count",
     "E4M3_MAX", "IDX_HEADS", "IDX_DIM", "MLA_HEADS", "D_QK", "D_V", "PAGE",
 ]
 
@@ -180,10 +180,6 @@ def topk_row(scores_row, n: int, k: int) -> np.ndarray:
     return out
 
 
-def topk_rows(scores, row_len, k: int) -> np.ndarray:
-    return np.stack([topk_row(scores[t], int(row_len[t]), k) for t in range(scores.shape[0])])
-
-
 # ----------------------------------------------------------------------------- attention
 
 
@@ -225,32 +221,37 @@ def dense_causal_attention_row(Q, KV_prefix, softmax_scale: float):
     return out, lse
 
 
-def sparse_mla(Q, KV, idx_rows, softmax_scale, rows=None, q_rows_per_idx_row: int = 1):
-    """Sparse MLA for several query rows; query row r uses idx_rows[r // q_rows_per_idx_row]."""
-    rows = range(Q.shape[0]) if rows is None else rows
-    O, L = {}, {}
-    for r in rows:
-        O[r], L[r] = sparse_mla_row(Q[r], KV, idx_rows[r // q_rows_per_idx_row], softmax_scale)
-    return O, L
-
-
 # ----------------------------------------------------------------------------- group / schedule
 
 
-def group_prefill(inp: dict, rows, fp8_indexer: bool = False, idx_override=None):
+def prefill_tables(inp: dict, fp8_indexer: bool = False) -> dict:
+    """The whole-sequence tables of a prefill group as fp64 values: the indexer keys (bf16, or
+    quantised per token to e4m3 and dequantised, R5) and each layer's latent KV rows.
+
+    Computed once per input set; :func:`group_prefill` takes them so that a call over a few
+    query rows does only those rows' work."""
+    if fp8_indexer:
+        k8, sk = quantize_e4m3_rows(inp["k_idx"], IDX_DIM)
+        keys = e4m3_to_f64(k8) * sk.reshape(-1, 1)
+    else:
+        keys = bf16_to_f64(inp["k_idx"])
+    return {"fp8_indexer": fp8_indexer, "keys": keys, "KV": [bf16_to_f64(x) for x in inp["KV"]]}
+
+
+def group_prefill(inp: dict, rows, fp8_indexer: bool = False, idx_override=None, tables=None):
     """One IndexShare group in causal prefill for the listed query rows (R1-R6).
 
     inp holds numpy arrays as built by the input generator (bf16 as uint16 bits):
     q_idx [L,32,128], w [L,32], k_idx [L,128], Q[l] [L,64,576], KV[l] [L,576].
-    Layer 0 is Full: scores + Top-k; layers 1.. reuse its indices.
+    Layer 0 is Full: scores + Top-k; layers 1.. reuse its indices.  ``tables`` (from
+    :func:`prefill_tables` with the same ``fp8_indexer``) skips the whole-table conversions.
     Returns {"idx": {t: [k]}, "O": [ {t: [64,512]} per layer ], "lse": [...]}."""
     L, k = inp["L"], inp["k"]
     rows = list(rows)
-    if fp8_indexer:
-        k8, sk = quantize_e4m3_rows(inp["k_idx"], IDX_DIM)
-        kv = e4m3_to_f64(k8) * sk.reshape(-1, 1)
-    else:
-        kv = bf16_to_f64(inp["k_idx"])
+    if tables is None:
+        tables = prefill_tables(inp, fp8_indexer)
+    assert tables["fp8_indexer"] == fp8_indexer
+    kv = tables["keys"]
 
     def query(t):  # indexer query of row t (only the rows asked for are converted)
         if fp8_indexer:
@@ -269,7 +270,7 @@ def group_prefill(inp: dict, rows, fp8_indexer: bool = False, idx_override=None)
     outO, outL = [], []
     for l in range(len(inp["Q"])):
         Q = inp["Q"][l]
-        KVl = bf16_to_f64(inp["KV"][l])
+        KVl = tables["KV"][l]
         O, Ls = {}, {}
         for t in rows:
             O[t], Ls[t] = sparse_mla_row(bf16_to_f64(Q[t]), KVl, idx[t], inp["softmax_scale"])

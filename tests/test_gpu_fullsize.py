@@ -76,14 +76,16 @@ def test_fullsize_prefill_sampled_rows(name):
         sc = O.indexer_scores(qv, host["w"][t][None].astype(np.float64), kv, [t + 1])[0]
         check_topk_sets(idx[t], sc, t + 1, k)
     # attention on the GPU's own indices, every layer
-    ref = O.group_prefill(host, rows, fp8_indexer=spec.indexer_fp8, idx_override={t: idx[t] for t in rows})
+    tables = O.prefill_tables(host, spec.indexer_fp8)
+    ref = O.group_prefill(host, rows, fp8_indexer=spec.indexer_fp8, idx_override={t: idx[t] for t in rows},
+                          tables=tables)
     for l in range(4):
         o = {t: O.bf16_to_f64(host_bits(out[l][t])) for t in rows}
         for t in rows:
             ma, rl = attn_errors(o[t], ref["O"][l][t])
             assert ma <= 2e-2 and rl <= 5e-3, (name, l, t, ma, rl)
     if spec.indexer_fp8:   # end to end against the oracle's own selection on the same inputs
-        own = O.group_prefill(host, rows, fp8_indexer=True)
+        own = O.group_prefill(host, rows, fp8_indexer=True, tables=tables)
         num = den = 0.0
         for l in range(4):
             for t in rows:

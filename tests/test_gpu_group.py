@@ -3,8 +3,12 @@
 Covers the 512-token tiny prefill workload in full, a scaled FP8-indexer prefill, a
 scaled batched decode with MTP rows and paged FP8 caches (rows reusing row 0's Top-k, and
 rows taking their own), and the reuse-handle rules.
-Tolerances as in test_gpu_kernels.py; the FP8 indexer path also checks end-to-end
-relative L2 <= 3e-2 against the oracle run on unquantised bf16 inputs.
+Tolerances as in test_gpu_kernels.py.  The FP8 indexer path is checked twice: its Top-k sets
+exactly (up to the tolerance band) against the oracle's scores on the dequantised e4m3 inputs,
+and its attention outputs end to end, relative L2 <= 3e-2 over the sampled rows, against the
+oracle run on the same inputs with its own e4m3 quantisation and its own selection.  (Against
+the unquantised bf16 inputs no e4m3 scheme can meet 3e-2: quantisation alone changes about 2%
+of each Top-2048 set, which moves the outputs by about 18%.)
 """
 import math
 

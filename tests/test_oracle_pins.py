@@ -380,3 +380,172 @@ def test_planted_cache_write_mistakes_are_caught(old, new):
     bad = _mutant(O.cache_write_e4m3, old, new)
     with pytest.raises(AssertionError):
         test_cache_write_fills_the_slots_paged_rows_reads(bad)
+
+
+# ----------------------------------------------------------------------------- group selection (Full layer)
+#
+# The Full layer's selection inside the group functions is pinned against scores computed
+# here by plain loops over heads, dims and the causal candidates s <= t (decode: s < N_b), with
+# FP8 values produced by torch's own e4m3 conversion at the per-vector scale amax / 448, and
+# the rank rule of _rank_select.  The inputs give the 32 heads of a query, and the keys of
+# different tokens, magnitudes several octaves apart, so that a scale taken per token instead
+# of per head, or a key scale applied to the wrong token, changes the selected sets.
+
+
+def _torch_e4m3_values(x32, vec_len):
+    """Per-vector e4m3 round trip through torch's float8_e4m3fn conversion: scale = amax / 448
+    in fp32 (1 when amax = 0), x / scale saturated to +-448, returned as fp64 values."""
+    x = torch.from_numpy(np.ascontiguousarray(x32, dtype=np.float32)).reshape(-1, vec_len)
+    amax = x.abs().amax(dim=1)
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    v = (x / scale[:, None]).clamp(-448.0, 448.0)
+    back = v.to(torch.float8_e4m3fn).to(torch.float64) * scale.to(torch.float64)[:, None]
+    return back.reshape(np.shape(x32)).numpy()
+
+
+def _loop_scores(q, w, keys, n):
+    """I[s] = sum_h w[h] * max(0, sum_d q[h,d] * keys[s,d]) for s < n, by plain loops."""
+    out = []
+    for s in range(n):
+        tot = 0.0
+        for h in range(q.shape[0]):
+            x = math.fsum(float(q[h, d]) * float(keys[s, d]) for d in range(q.shape[1]))
+            tot += float(w[h]) * max(0.0, x)
+        out.append(tot)
+    return np.array(out)
+
+
+def _octave_prefill_inputs(seed=21, L=40, k=6):
+    """Tiny prefill group whose indexer query heads and key tokens span many octaves (the head
+    weights undo the query heads' spread, so that every head moves the scores)."""
+    from synth.generators import bf16_bits_np
+    rng = np.random.default_rng(seed)
+    q = rng.normal(size=(L, 32, 128)) * (2.0 ** (-np.arange(32) / 2.0))[None, :, None]
+    kk = rng.normal(size=(L, 128)) * (2.0 ** rng.integers(-6, 7, size=L))[:, None]
+    inp = make_prefill(PrefillSpec("oct", L=L, k=k, n_layers=1, seed=seed))
+    inp["q_idx"] = bf16_bits_np(q)
+    inp["k_idx"] = bf16_bits_np(kk)
+    inp["w"] = (inp["w"] * (2.0 ** (np.arange(32) / 2.0))[None, :]).astype(np.float32)  # every head counts
+    return inp
+
+
+def _check_prefill_selection(fn, fp8):
+    inp = _octave_prefill_inputs()
+    L, k = inp["L"], inp["k"]
+    rows = list(range(L))
+    g = fn(inp, rows, fp8_indexer=fp8)
+    qv = O.bf16_to_f64(inp["q_idx"])
+    kv = O.bf16_to_f64(inp["k_idx"])
+    if fp8:
+        qv = _torch_e4m3_values(qv.astype(np.float32), 128)     # one scale per (token, head)
+        kv = _torch_e4m3_values(kv.astype(np.float32), 128)     # one scale per key token
+    for t in rows:
+        sc = _loop_scores(qv[t], inp["w"][t], kv, t + 1)        # candidates s = 0 .. t
+        got = g["idx"][t]
+        assert set(int(i) for i in got if i >= 0) == _rank_select(sc, t + 1, k), t
+        assert (got[min(k, t + 1):] == -1).all()
+
+
+def test_group_prefill_selection_is_the_loop_definition(fn=None):
+    _check_prefill_selection(fn or O.group_prefill, fp8=False)
+
+
+def test_group_prefill_fp8_selection_is_the_loop_definition(fn=None):
+    _check_prefill_selection(fn or O.group_prefill, fp8=True)
+
+
+def test_prefill_tables_reuse_gives_the_same_group():
+    inp = _octave_prefill_inputs(seed=4)
+    for fp8 in (False, True):
+        tab = O.prefill_tables(inp, fp8)
+        a = O.group_prefill(inp, [3, 17, 39], fp8_indexer=fp8)
+        b = O.group_prefill(inp, [3, 17, 39], fp8_indexer=fp8, tables=tab)
+        for t in (3, 17, 39):
+            assert np.array_equal(a["idx"][t], b["idx"][t]) and np.array_equal(a["O"][0][t], b["O"][0][t])
+
+
+def _octave_decode_inputs(seed=12):
+    """Tiny decode batch whose query heads span many octaves; key pool as generated."""
+    from synth.generators import bf16_bits_np
+    spec = DecodeSpec("oct", batch=3, ctx_lo=70, ctx_hi=200, rows_per_seq=2, k=12, n_layers=1, seed=seed)
+    inp = make_decode(spec)
+    rng = np.random.default_rng(seed)
+    q = rng.normal(size=(3, 32, 128)) * (2.0 ** (-np.arange(32) / 2.0))[None, :, None]
+    inp["q_idx"] = bf16_bits_np(q)
+    inp["w"] = (inp["w"] * (2.0 ** (np.arange(32) / 2.0))[None, :]).astype(np.float32)  # every head counts
+    return inp
+
+
+def _dense_cache_by_pages(pool, scale, bt, b, n):
+    """Sequence b's first n cache rows, read page by page of its block table (torch e4m3 decode)."""
+    rows = np.zeros((n, pool.shape[2]))
+    vals = torch.from_numpy(np.ascontiguousarray(pool)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for lp in range((n + 63) // 64):
+        p = int(bt[b][lp])
+        for j in range(64):
+            s = lp * 64 + j
+            if s < n:
+                rows[s] = vals[p, j] * float(scale[p, j])
+    return rows
+
+
+def test_group_decode_selection_is_the_loop_definition(fn=None):
+    fn = fn or O.group_decode
+    inp = _octave_decode_inputs()
+    g = fn(inp)
+    qv = _torch_e4m3_values(O.bf16_to_f64(inp["q_idx"]).astype(np.float32), 128)
+    for b in range(len(inp["ctx"])):
+        n = int(inp["ctx"][b])
+        keys = _dense_cache_by_pages(inp["idx_keys"], inp["idx_key_scale"], inp["block_table"], b, n)
+        sc = _loop_scores(qv[b], inp["w"][b], keys, n)          # candidates s = 0 .. N_b - 1
+        got = g["idx"][b]
+        assert set(int(i) for i in got if i >= 0) == _rank_select(sc, n, inp["k"]), b
+
+
+@pytest.mark.parametrize("edits", [
+    [('quantize_e4m3_rows(np.asarray(inp["q_idx"][t])[None], IDX_DIM)',
+      'quantize_e4m3_rows(np.asarray(inp["q_idx"][t])[None], IDX_HEADS * IDX_DIM)'),
+     ("sq.reshape(1, IDX_HEADS, 1)", "sq.reshape(1, 1, 1)")],          # one query scale per token, not per head
+    [("[t + 1])[0]", "[t])[0]")],                                       # query t scores only s < t
+    [("topk_row(sc, t + 1, k)", "topk_row(sc, t, k)")],                 # query t selects among s < t
+    [('wt = np.asarray(inp["w"][t]', 'wt = np.asarray(inp["w"][0]')],  # the first row's head weights
+])
+def test_planted_group_prefill_fp8_mistakes_are_caught(edits):
+    bad = _mutant_src(O.group_prefill, edits)
+    with pytest.raises(AssertionError):
+        test_group_prefill_fp8_selection_is_the_loop_definition(bad)
+
+
+@pytest.mark.parametrize("old,new", [
+    ('keys = e4m3_to_f64(k8) * sk.reshape(-1, 1)', 'keys = e4m3_to_f64(k8) * sk[::-1].reshape(-1, 1)'),  # wrong token's scale
+    ('keys = e4m3_to_f64(k8) * sk.reshape(-1, 1)', 'keys = e4m3_to_f64(k8) * 1.0'),                      # scale dropped
+])
+def test_planted_key_scale_mistakes_are_caught(old, new):
+    bad_tables = _mutant(O.prefill_tables, old, new)
+
+    def bad(inp, rows, fp8_indexer=False):
+        return O.group_prefill(inp, rows, fp8_indexer, tables=bad_tables(inp, fp8_indexer))
+    with pytest.raises(AssertionError):
+        test_group_prefill_fp8_selection_is_the_loop_definition(bad)
+
+
+@pytest.mark.parametrize("edits", [
+    [('quantize_e4m3_rows(inp["q_idx"], IDX_DIM)', 'quantize_e4m3_rows(inp["q_idx"], IDX_HEADS * IDX_DIM)'),
+     ("sq.reshape(-1, IDX_HEADS, 1)", "sq.reshape(-1, 1, 1)")],              # per-token query scale
+    [("w[b:b + 1], keys, [n])", "w[b:b + 1], keys, [n - 1])")],            # the newest token left out
+    [('inp["idx_key_scale"], bt[b], n)', 'inp["idx_key_scale"], bt[0], n)')],  # first sequence's pages
+])
+def test_planted_group_decode_mistakes_are_caught(edits):
+    bad = _mutant_src(O.group_decode, edits)
+    with pytest.raises(AssertionError):
+        test_group_decode_selection_is_the_loop_definition(bad)
+
+
+def _mutant_src(fn, edits):
+    src = inspect.getsource(fn)
+    for old, new in edits:
+        assert old in src, (old, fn.__name__)
+        src = src.replace(old, new)
+    ns = dict(vars(O))
+    exec(compile(src, "<mutant>", "exec"), ns)
+    return ns[fn.__name__]
