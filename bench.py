@@ -1,21 +1,29 @@
 #!/usr/bin/env python
-"""Benchmark of one DSA + IndexShare step on B200: query tokens/s per IndexShare group.
+"""Benchmark of the DSA + IndexShare step on B200: query tokens/s per IndexShare group.
 
-A step is one IndexShare group on one batch of synthetic input: the Full layer's indexer
-scores + Top-k into the reuse handle, then sparse MLA for the Full layer and its 3 Shared
-layers.  Default workload: causal prefill of 32,768 tokens, Top-2048, bf16, AR(1)-drifting
-indexer keys.  Inputs are generated on the device by the seeded generator before timing.
+A step is one pass of the whole hot path over one batch of synthetic input: the Full layer's
+indexer scores + Top-k into the reuse handle, then sparse MLA for the Full layer and its 3
+Shared layers (decode: the current token's rows are first written into the paged FP8 caches,
+and a 78-layer step runs the 21 groups of the schedule).  Inputs are generated on the device by
+the seeded generator before timing.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|all] [--impl reference]
 
-One JSON line is printed by rank 0.  Multi-GPU (torchrun): every rank runs its own
-independent group (weak scaling, no collective on the data path); the time is the max over
-ranks of the CUDA-event time.  ``--impl reference`` times the fp64 CPU oracle on a bounded
-sample of the same workload (rank 0 only).
+Default (``all``): the headline line is causal prefill of 131,072 tokens with the FP8 indexer
+(the largest single-GPU prefill workload), timed over exactly K steps; the same process then
+measures the other workloads (512-token tiny prefill, 32K bf16 prefill, batch-32 decode with 4
+MTP draft rows and without, 1M-token 78-layer decode) and reports each under ``workloads``, each
+timed over at least one second of steps so that the clock sampler sees it.
+
+One JSON line is printed by rank 0.  Multi-GPU (torchrun): every rank runs its own independent
+problem (weak scaling, no collective on the data path); the time is the max over ranks of the
+CUDA-event time.  ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+headline workload (rank 0 only).
 """
 from __future__ import annotations
 
 import argparse
+import gc
 import json
 import math
 import os
@@ -29,6 +37,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "query tokens/s per IndexShare group"
 UNIT = "query tokens/s"
+HEADLINE = "prefill_128k_fp8"
+SUB_WORKLOADS = ["tiny_prefill", "prefill_32k", "decode_b32_mtp4", "decode_b32_d0", "decode_1m_mtp5"]
+ALL_WORKLOADS = ["tiny_prefill", "prefill_32k", "prefill_128k_fp8", "decode_b32_mtp4", "decode_b32_d0",
+                 "decode_b32_mtp4_verify", "decode_1m_mtp5"]
 
 # sparse_mla_kernel<bf16>, L=8,192 prefill launch (8,192 query rows): ncu measured 672.8 MB read
 # + 510.4 MB written = 144,436 B per query row (queries 73,728 B in, outputs 65,536 B out, the
@@ -36,25 +48,24 @@ UNIT = "query tokens/s"
 MLA_DRAM_BYTES_PER_ROW_BF16 = (672.798720e6 + 510.417920e6) / 8192
 
 
-
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
-    p.add_argument("--workload", default="prefill_32k",
-                   choices=["tiny_prefill", "prefill_32k", "prefill_128k_fp8", "decode_b32_mtp4", "decode_b32_d0",
-                            "decode_b32_mtp4_verify",
-                            "decode_1m_mtp5"])
+    p.add_argument("--workload", default="all", choices=["all"] + ALL_WORKLOADS)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     p.add_argument("--ref-seconds", type=float, default=150.0, help="reference arm total budget")
     p.add_argument("--seq-len", type=int, default=None, help="override L of a prefill workload (profiling)")
+    p.add_argument("--min-timed-s", type=float, default=1.0,
+                   help="least timed seconds of each workload under 'workloads' (clock samples)")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-sub", action="store_true", help="headline workload only")
     p.add_argument("--graph", choices=["auto", "on", "off"], default="auto",
                    help="replay each step as one captured CUDA graph (auto: decode workloads)")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    return p.parse_args()
+    return p.parse_args(argv)
 
 
 # ----------------------------------------------------------------------------- distributed
@@ -95,7 +106,7 @@ def max_over_ranks(x, ws):
 
 
 def job_throughput(tokens_per_rank, steps, ws, total_ms_max):
-    """Whole-job tokens/s: every rank processes its own group per step (weak scaling)."""
+    """Whole-job tokens/s: every rank processes its own problem per step (weak scaling)."""
     return tokens_per_rank * ws * steps / (total_ms_max / 1e3)
 
 
@@ -111,7 +122,8 @@ def workload_config(name, seq_len=None):
     if name.startswith("decode"):
         cfg = {"workload": name, "batch": spec.batch, "context": f"U[{spec.ctx_lo},{spec.ctx_hi}]",
                "rows_per_seq": spec.rows_per_seq, "k": spec.k, "layers": spec.n_layers,
-               "cache": "paged e4m3 (64-token pages), device-resident across steps", "indexer": "e4m3",
+               "cache": "paged e4m3 (64-token pages), device-resident across steps; the step writes its "
+                        "current token's rows first (one launch per pool)", "indexer": "e4m3",
                "topk": "one per query row" if spec.topk_per_row else "row 0's, reused by the draft rows"}
         if spec.n_layers > 4:
             cfg["schedule"] = "Full at layers 0, 1, 2+4g; 21 groups per step"
@@ -119,6 +131,10 @@ def workload_config(name, seq_len=None):
     return spec, {"workload": name, "seq_len": spec.L, "k": spec.k, "layers_per_group": spec.n_layers,
                   "indexer": "e4m3" if spec.indexer_fp8 else "bf16", "latent_kv": "bf16 [L,576]",
                   "heads": 64, "indexer_heads": 32}
+
+
+def workload_dtype(name):
+    return "bf16" if name in ("tiny_prefill", "prefill_32k") else "bf16+e4m3"
 
 
 def algorithmic_counts(spec, ctx=None):
@@ -148,12 +164,13 @@ class Workload:
     def __init__(self, spec, name, dev):
         import torch
         import long_context_sparse_11_b200 as dsa
-        from synth import make_prefill, make_decode, make_decode_indexer
+        from synth import make_prefill, make_decode, make_decode_indexer, make_decode_new_tokens
         self.name, self.spec = name, spec
-        self.groups, self.step_inputs, self.layers_per_group = [], [], []
+        self.groups, self.step_inputs, self.layers_per_group, self.writes = [], [], [], []
         if name.startswith("decode"):
             inp = make_decode(spec, device=dev)
             self.inp = inp
+            B = len(inp["ctx"])
             ctx_d = torch.from_numpy(inp["ctx"].astype("int32")).to(dev)
             bt_d = torch.from_numpy(inp["block_table"]).to(dev)
             # per-row Top-k: every query row is its own entry of the views (same pages, same length)
@@ -162,8 +179,14 @@ class Workload:
                    for l in range(spec.n_layers)]
             fulls = [l for l in range(spec.n_layers) if dsa.layer_is_full(l)] if spec.n_layers > 4 else [0]
             ends = fulls[1:] + [spec.n_layers]
+            new = make_decode_new_tokens(spec, B, range(spec.n_layers), fulls, device=dev)
+            self.pos = torch.from_numpy((inp["ctx"] - 1).astype("int32")).to(dev)   # the current token
+            self.bt = bt_d
+            for l in range(spec.n_layers):
+                self.writes.append((new["kv"][l], inp["KV"][l], inp["KV_scale"][l]))
             for f, e in zip(fulls, ends):
-                ind = inp if f == 0 else make_decode_indexer(spec, f, inp["n_pages"], len(inp["ctx"]), dev)
+                ind = inp if f == 0 else make_decode_indexer(spec, f, inp["n_pages"], B, dev)
+                self.writes.append((new["key"][f], ind["idx_keys"], ind["idx_key_scale"]))
                 keys = dsa.paged_view(ind["idx_keys"], ind["idx_key_scale"], bt_d, ctx_d, rows_per_seq=rows)
                 g = dsa.IndexShareGroup(ind["q_idx"], ind["w"], keys, spec.k, inp["Q"][f:e], kvs[f:e],
                                         inp["softmax_scale"], indexer_dtype=dsa.DSA_E4M3,
@@ -172,6 +195,7 @@ class Workload:
                 self.layers_per_group.append(e - f)
                 # a decode step's new inputs: the indexer query and weights, the MLA query rows
                 self.step_inputs += [ind["q_idx"], ind["w"]] + list(inp["Q"][f:e])
+            self.step_inputs += [x for x, _, _ in self.writes]     # and the current token's rows
             self.counts = algorithmic_counts(spec, inp["ctx"])
         else:
             inp = make_prefill(spec, device=dev)
@@ -190,6 +214,9 @@ class Workload:
         return [t for g in self.groups for t in g.out + g.lse]
 
     def forward(self):
+        import long_context_sparse_11_b200 as dsa
+        for x, pool, scale in self.writes:
+            dsa.cache_write_e4m3(x, self.pos, self.bt, pool, scale)
         for g in self.groups:
             g.forward()
 
@@ -231,6 +258,36 @@ def indexer_alone(wl, spec, dev, stream):
     return ms, (L + R - 1) // R
 
 
+def independent_full_layers(wl, spec, stream, flush, reps=3):
+    """The same sequence run as 4 independent Full layers: each layer its own group call of one
+    layer (its own a1-a4 on the indexer inputs, then its own a6), back to back on the stream."""
+    import torch
+    import long_context_sparse_11_b200 as dsa
+    inp = wl.inp
+    groups = [dsa.IndexShareGroup(inp["q_idx"], inp["w"], dsa.dense_view(inp["k_idx"]), spec.k, [inp["Q"][l]],
+                                  [dsa.dense_view(inp["KV"][l])], inp["softmax_scale"],
+                                  indexer_dtype=dsa.DSA_E4M3 if spec.indexer_fp8 else dsa.DSA_BF16)
+              for l in range(spec.n_layers)]
+    for g in groups:
+        g.forward()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for g in groups:
+            g.forward()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    dsa.sync_status()
+    del groups
+    gc.collect()
+    torch.cuda.empty_cache()
+    return statistics.mean(times)
+
+
 # ----------------------------------------------------------------------------- clocks
 
 
@@ -262,17 +319,6 @@ class ClockSampler:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
             self.lines = [l for l in out.splitlines() if l.strip()]
-        self.after = False
-        if self.proc is not None and not self.lines:
-            # a timed region shorter than one sampling period: one reading right after it
-            try:
-                out = subprocess.run(["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
-                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
-                                     timeout=10).stdout
-                self.lines = [l for l in out.splitlines() if l.strip()]
-                self.after = bool(self.lines)
-            except (OSError, subprocess.TimeoutExpired):
-                pass
 
     def summary(self):
         sm, mx, reasons = [], None, set()
@@ -289,11 +335,8 @@ class ClockSampler:
             for n, v in zip(names, f[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-               "samples": 0 if getattr(self, "after", False) else len(sm)}
-        if getattr(self, "after", False):
-            out["read_after_timed_region"] = True   # the region was shorter than the 100 ms period
-        return out
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
 
 
 def gpu_smi_id(dev_index):
@@ -316,8 +359,9 @@ def measured_peaks():
 # ----------------------------------------------------------------------------- CPU oracle sample
 
 
-def oracle_rows_per_second(spec, name, inp, budget_s, seed_rows=0):
-    """Time the fp64 oracle on a bounded sample of rows of the same workload (host cores)."""
+def host_inputs(spec, name, inp):
+    """The oracle's view of a workload: host arrays (bf16 as uint16 bits) and, for prefill, the
+    whole-sequence fp64 tables converted once, so that a timed call does only its rows' work."""
     import numpy as np
     import oracle.dsa_oracle as O
     import torch
@@ -327,13 +371,27 @@ def oracle_rows_per_second(spec, name, inp, budget_s, seed_rows=0):
 
     if name.startswith("decode"):
         nl = 4 if len(inp["Q"]) <= 4 else 1   # the first IndexShare group (layers 0..3, or layer 0 of 78)
-        host = {"ctx": inp["ctx"], "block_table": inp["block_table"], "k": spec.k, "rows_per_seq": spec.rows_per_seq,
+        return {"ctx": inp["ctx"], "block_table": inp["block_table"], "k": spec.k, "rows_per_seq": spec.rows_per_seq,
                 "softmax_scale": spec.softmax_scale, "q_idx": host_bits(inp["q_idx"]), "w": inp["w"].cpu().numpy(),
                 "idx_keys": inp["idx_keys"].cpu().numpy(), "idx_key_scale": inp["idx_key_scale"].cpu().numpy(),
                 "Q": [host_bits(q) for q in inp["Q"][:nl]], "KV": [x.cpu().numpy() for x in inp["KV"][:nl]],
-                "KV_scale": [x.cpu().numpy() for x in inp["KV_scale"][:nl]]}
+                "KV_scale": [x.cpu().numpy() for x in inp["KV_scale"][:nl]], "n_layers_timed": nl}
+    host = {"L": spec.L, "k": spec.k, "softmax_scale": spec.softmax_scale, "k_idx": host_bits(inp["k_idx"]),
+            "q_idx": _LazyRows(inp["q_idx"]), "w": _LazyRows(inp["w"], bf16=False),
+            "Q": [_LazyRows(q) for q in inp["Q"]], "KV": [host_bits(x) for x in inp["KV"]]}
+    host["tables"] = O.prefill_tables(host, spec.indexer_fp8)
+    return host
+
+
+def oracle_rows_per_second(spec, name, host, budget_s, seed_rows=0):
+    """Time the fp64 oracle on a bounded sample of rows of the same workload (host cores).
+    Returns (rows per second, sample description, seconds)."""
+    import numpy as np
+    import oracle.dsa_oracle as O
+    if name.startswith("decode"):
+        nl = host["n_layers_timed"]
         policy = O.group_decode_per_row if spec.topk_per_row else O.group_decode
-        order = list(np.random.default_rng(seed_rows).permutation(len(inp["ctx"])))
+        order = list(np.random.default_rng(seed_rows).permutation(len(host["ctx"])))
         done, t0 = 0, time.perf_counter()
         while order and time.perf_counter() - t0 < budget_s:
             policy(host, seqs=[order.pop()])
@@ -342,21 +400,16 @@ def oracle_rows_per_second(spec, name, inp, budget_s, seed_rows=0):
         return done / el, (f"{done // spec.rows_per_seq} whole sequences (all {spec.rows_per_seq} rows, indexer, "
                            f"Top-k and {nl} layer(s) of the first group)"), el
     L = spec.L
-    host = {"L": L, "k": spec.k, "softmax_scale": spec.softmax_scale, "k_idx": host_bits(inp["k_idx"]),
-            "q_idx": _LazyRows(inp["q_idx"]), "w": _LazyRows(inp["w"], bf16=False),
-            "Q": [_LazyRows(q) for q in inp["Q"]], "KV": [host_bits(x) for x in inp["KV"]]}
     rng = np.random.default_rng(seed_rows)
-    # one oracle call over a batch of uniformly drawn rows, sized from a short calibration
-    n, el = 2, 0.0
-    for _ in range(6):
-        rows = sorted(int(r) for r in rng.integers(0, L, size=n))
-        t0 = time.perf_counter()
-        O.group_prefill(host, rows, fp8_indexer=spec.indexer_fp8)
-        el = time.perf_counter() - t0
-        if el >= 0.5 * budget_s:
-            break
-        n = max(n + 1, int(n * min(8.0, budget_s / max(el, 1e-3))))
-    return n / el, f"{n} uniformly drawn query rows in one oracle call (indexer + Top-k + 4 layers each)", el
+    rows_done, el = 0, 0.0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s or rows_done == 0:
+        rows = sorted(int(r) for r in rng.integers(0, L, size=2))
+        O.group_prefill(host, rows, fp8_indexer=spec.indexer_fp8, tables=host["tables"])
+        rows_done += 2
+    el = time.perf_counter() - t0
+    return rows_done / el, (f"{rows_done} uniformly drawn query rows, 2 per oracle call (indexer + Top-k + "
+                            f"{len(host['Q'])} layers each; whole-sequence tables converted once, untimed)"), el
 
 
 class _LazyRows:
@@ -375,32 +428,34 @@ class _LazyRows:
 
 
 def cpu_cores():
+    """(threads the oracle's BLAS calls use, note): the oracle is numpy fp64 in one process."""
     try:
         from threadpoolctl import threadpool_info
         th = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
         th = 1
-    return max(1, min(th, len(os.sched_getaffinity(0))))
+    th = max(1, min(th, len(os.sched_getaffinity(0))))
+    return th, (f"numpy fp64 in one process: the loop over rows runs on one core, its matrix products "
+                f"(BLAS) on {th} threads; {len(os.sched_getaffinity(0))} host cores available")
 
 
-# ----------------------------------------------------------------------------- arms
+# ----------------------------------------------------------------------------- our arm
 
 
-def run_ours(args, ws, rank, local):
+def measure(name, args, ws, rank, local, headline):
+    """Build one workload, time it and return its measurement (rank 0's view of the max over ranks)."""
     import ctypes
     import torch
     import long_context_sparse_11_b200 as dsa
-    from long_context_sparse_11_b200.build import build
 
-    build()
     lib = dsa.load()
     dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    spec, cfg = workload_config(args.workload, args.seq_len)
-    wl = Workload(spec, args.workload, dev)
+    spec, cfg = workload_config(name, args.seq_len if headline else None)
+    wl = Workload(spec, name, dev)
     counts = wl.counts
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.int32, device=dev)   # 1 GiB > 126 MB L2
+    decode = name.startswith("decode")
 
     # trace events per group: the Full layer's a1-a4 phase and each layer's sparse MLA launch
     # (recorded once so that torch creates the CUDA events before their handles are passed on)
@@ -424,12 +479,14 @@ def run_ours(args, ws, rank, local):
     dsa.sync_status()
     torch.cuda.synchronize()
     n0 = lib.dsa_launch_count()
+    t0 = time.perf_counter()
     step(False)
     torch.cuda.synchronize()
+    est_ms = 1e3 * (time.perf_counter() - t0)
     launches_per_step = lib.dsa_launch_count() - n0
 
     # many short kernels (decode): the step is captured once as a CUDA graph and replayed
-    use_graph = args.graph == "on" or (args.graph == "auto" and args.workload.startswith("decode"))
+    use_graph = args.graph == "on" or (args.graph == "auto" and decode)
     graph = None
     if use_graph:
         graph = torch.cuda.CUDAGraph()
@@ -438,12 +495,19 @@ def run_ours(args, ws, rank, local):
         graph.replay()
         torch.cuda.synchronize()
         dsa.sync_status()
+        t0 = time.perf_counter()
+        for _ in range(5):
+            graph.replay()
+        torch.cuda.synchronize()
+        est_ms = 1e3 * (time.perf_counter() - t0) / 5
 
     def run_step():
         if graph is not None:
             graph.replay()
         else:
             wl.forward()
+
+    mla_ms, idx_ms = [], []
 
     def timed_steps(n, traced):
         out = []
@@ -457,32 +521,38 @@ def run_ours(args, ws, rank, local):
             else:
                 run_step()
             s1.record(stream)
-            s1.synchronize()
-            out.append(s0.elapsed_time(s1))
+            if traced or n <= 64:
+                s1.synchronize()
+            out.append((s0, s1))
             if traced:
                 for evs, nl in zip(traces, wl.layers_per_group):
                     idx_ms.append(evs[0].elapsed_time(evs[1]))
                     mla_ms.extend(evs[2 + 2 * l].elapsed_time(evs[3 + 2 * l]) for l in range(nl))
-        return out
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in out]
 
-    mla_ms, idx_ms = [], []
+    # the headline times exactly K steps; the other workloads at least min_timed_s of steps
+    steps = args.steps
+    if not headline:
+        steps = max(steps, int(math.ceil(1e3 * args.min_timed_s / max(est_ms, 1e-3))))
+        steps = int(max_over_ranks(float(steps), ws))
     torch.cuda.synchronize()
     barrier(ws)                                             # all ranks start the timed steps together
     with ClockSampler(gpu_smi_id(local)) as clk:
         # eager steps carry the library's phase events; graph replays are timed on their own and
-        # the phase split comes from as many eager steps run afterwards
-        t_steps = timed_steps(args.steps, traced=graph is None)
+        # the phase split comes from eager steps run afterwards
+        t_steps = timed_steps(steps, traced=graph is None)
     torch.cuda.synchronize()
     barrier(ws)
     if graph is not None:
-        timed_steps(args.steps, traced=True)
+        timed_steps(min(steps, 20), traced=True)
         torch.cuda.synchronize()
-    launches = launches_per_step * args.steps
+    launches = launches_per_step * steps
     dsa.sync_status()
     total_ms = max_over_ranks(sum(t_steps), ws)
-    ms_per_step = total_ms / args.steps
+    ms_per_step = total_ms / steps
     n_groups = len(wl.groups)
-    value = job_throughput(counts["tokens"] * n_groups, args.steps, ws, total_ms)
+    value = job_throughput(counts["tokens"] * n_groups, steps, ws, total_ms)
     clocks = clk.summary()
 
     hbm, bf16_peak, peak_kind = measured_peaks()
@@ -490,7 +560,7 @@ def run_ours(args, ws, rank, local):
     idx_avg = statistics.mean(idx_ms)
     mla_tf = counts["mla_flops_per_layer"] / (mla_avg / 1e3) / 1e12
     traffic = None
-    if not args.workload.startswith("decode"):
+    if not decode:
         # DRAM bytes (read + write) of one bf16 launch grow with the query rows (queries in,
         # outputs out; the latent rows stay in L2): measured by ncu at 8,192 rows, scaled.
         traffic = {"bytes_per_launch": round(MLA_DRAM_BYTES_PER_ROW_BF16 * counts["mla_rows"]),
@@ -528,10 +598,9 @@ def run_ours(args, ws, rank, local):
             phases["mla_roofline"] = mla_roof
     if n_groups > 1:
         phases["step_ms_all_layers"] = round(ms_per_step, 4)
-    if not args.workload.startswith("decode"):
+    if not decode:
         # the indexer kernel alone against the tensor peak of its input type (e4m3: the measured
-        # bf16 peak x 2, the nominal fp8 / bf16 ratio), and the IndexShare group against four
-        # independent full layers (each with its own a1-a4), from the same phase timings
+        # bf16 peak x 2, the nominal fp8 / bf16 ratio)
         ia_ms, ia_launches = indexer_alone(wl, wl.spec, dev, stream)
         ia_tf = counts["indexer_flops"] / (ia_ms / 1e3) / 1e12
         ia_peak = bf16_peak * (2.0 if wl.spec.indexer_fp8 else 1.0)
@@ -539,12 +608,13 @@ def run_ours(args, ws, rank, local):
                                    "peak": round(ia_peak, 1), "frac": round(ia_tf / ia_peak, 4),
                                    "peak_source": f"{peak_kind} bf16 dense (burst)" +
                                    (" x 2 (fp8 / bf16 nominal)" if wl.spec.indexer_fp8 else "")}
-        nl = wl.layers_per_group[0]
-        group_ms = idx_avg + nl * mla_avg
-        full_ms = nl * (idx_avg + mla_avg)
+        # the IndexShare group against the same sequence run as 4 independent Full layers, both timed
+        full_ms = independent_full_layers(wl, wl.spec, stream, flush)
         phases["indexshare_vs_independent_full_layers"] = {
-            "group_ms": round(group_ms, 3), "independent_full_layers_ms": round(full_ms, 3),
-            "ratio": round(group_ms / full_ms, 4)}
+            "group_ms": round(ms_per_step, 3), "independent_full_layers_ms": round(full_ms, 3),
+            "ratio": round(ms_per_step / full_ms, 4),
+            "how": "both timed with CUDA events, L2 flushed before each; the 4 independent layers are 4 "
+                   "one-layer group calls that each run their own a1-a4 and a6"}
 
     def make_twin():
         """A second set of device inputs/outputs (the same seeded data), so that one step's upload
@@ -552,7 +622,7 @@ def run_ours(args, ws, rank, local):
         free, _ = torch.cuda.mem_get_info()
         if free < 1.25 * torch.cuda.memory_allocated() + (4 << 30):
             return None
-        wl2 = Workload(spec, args.workload, dev)
+        wl2 = Workload(spec, name, dev)
         wl2.forward()
         g2 = None
         if graph is not None:
@@ -567,20 +637,50 @@ def run_ours(args, ws, rank, local):
         e2e = run_e2e(args, wl, stream, ws, run_step, make_twin)
 
     cpu = None
-    if rank == 0 and not args.no_cpu_baseline and ws == 1:
-        v, sample, el = oracle_rows_per_second(spec, args.workload, wl.inp, args.cpu_seconds)
-        cpu = {"value": round(v, 3), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": sample,
-               "seconds": round(el, 1)}
+    if headline and rank == 0 and not args.no_cpu_baseline and ws == 1:
+        host = host_inputs(spec, name, wl.inp)
+        v, sample, el = oracle_rows_per_second(spec, name, host, args.cpu_seconds)
+        cores, note = cpu_cores()
+        cpu = {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+               "seconds": round(el, 1), "threads_note": note}
+        del host
+    cfg.update({"l2": "flushed (1 GiB write) between timed steps", "parallelism": f"replicas x{ws}",
+                "cuda_graph": graph is not None})
+    res = {"value": round(value, 1), "ms_per_step": round(ms_per_step, 4), "steps": steps, "warmup": args.warmup,
+           "dtype": workload_dtype(name), "config": cfg, "roofline": roofline, "phases": phases, "e2e": e2e,
+           "gpu_launches": launches, "clocks": clocks}
+    if cpu is not None:
+        res["cpu_baseline"] = cpu
+    del graph, wl, flush, traces, arrs
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args, ws, rank, local):
+    import torch
+    import long_context_sparse_11_b200 as dsa
+    from long_context_sparse_11_b200.build import build
+
+    build()
+    dsa.load()
+    torch.cuda.set_device(torch.device("cuda", local))
+    head_name = HEADLINE if args.workload == "all" else args.workload
+    head = measure(head_name, args, ws, rank, local, headline=True)
+    subs = {}
+    if args.workload == "all" and not args.no_sub:
+        for name in SUB_WORKLOADS:
+            subs[name] = measure(name, args, ws, rank, local, headline=False)
     if rank == 0:
-        cfg.update({"l2": "flushed (1 GiB write) between timed steps", "parallelism": f"replicas x{ws}",
-                    "cuda_graph": graph is not None})
-        dtype = "bf16" if args.workload.startswith("prefill_32k") or args.workload == "tiny_prefill" else "bf16+e4m3"
-        line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": dtype,
-                "data": "synthetic (seeded SplitMix64 normals)", "config": cfg,
-                "roofline": roofline, "phases": phases, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-                "clocks": clocks}
+        line = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": head["dtype"],
+                "data": "synthetic (seeded SplitMix64 normals)", "config": head["config"],
+                "roofline": head["roofline"], "phases": head["phases"], "cpu_baseline": head.get("cpu_baseline"),
+                "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"]}
+        if subs:
+            line["workloads"] = subs
         print(json.dumps(line), flush=True)
 
 
@@ -598,6 +698,8 @@ def run_e2e(args, wl, stream, ws, run_step, make_twin=None):
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
     steps = max(2, min(args.steps, 5))
+    if wl.name.startswith("decode"):
+        steps = 50                      # short steps: enough of them for a stable ratio
     sets = [(wl, run_step)]
     twin = make_twin() if make_twin is not None else None
     if twin is not None:
@@ -646,35 +748,44 @@ def run_e2e(args, wl, stream, ws, run_step, make_twin=None):
     ms = max_over_ranks(e0.elapsed_time(e1), ws)
     dsa.sync_status()
     tokens = wl.counts["tokens"] * len(wl.groups)
-    return {"value": round(tokens * ws * steps / (ms / 1e3), 1), "unit": UNIT,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 3), "device_buffer_sets": len(sets)}
+    res = {"value": round(tokens * ws * steps / (ms / 1e3), 1), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+           "ms_per_step": round(ms / steps, 3), "device_buffer_sets": len(sets)}
+    del host_in, host_out, sets, twin
+    gc.collect()
+    return res
+
+
+# ----------------------------------------------------------------------------- reference arm
 
 
 def run_reference(args, ws, rank):
-    """fp64 oracle on the host cores: each step a bounded sample of the same workload."""
+    """fp64 oracle on the host cores: each step a bounded sample of the same (headline) workload."""
     if rank != 0:
         return
     import torch
-    spec, cfg = workload_config(args.workload, args.seq_len)
+    name = HEADLINE if args.workload == "all" else args.workload
+    spec, cfg = workload_config(name, args.seq_len)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     from synth import make_prefill, make_decode
-    if args.workload.startswith("decode"):
+    if name.startswith("decode"):
         inp = make_decode(spec, device=dev)
     else:
         inp = make_prefill(spec, device=dev)
+    host = host_inputs(spec, name, inp)                    # untimed set-up: host copies, fp64 tables
     per_step = max(1.0, args.ref_seconds / (args.steps + args.warmup))
     for _ in range(args.warmup):
-        oracle_rows_per_second(spec, args.workload, inp, per_step, seed_rows=99)
+        oracle_rows_per_second(spec, name, host, per_step, seed_rows=99)
     tot_rows, tot_s, sample = 0.0, 0.0, ""
     for i in range(args.steps):
-        v, sample, el = oracle_rows_per_second(spec, args.workload, inp, per_step, seed_rows=i)
+        v, sample, el = oracle_rows_per_second(spec, name, host, per_step, seed_rows=i)
         tot_rows += v * el
         tot_s += el
     value = tot_rows / tot_s
     cfg.update({"parallelism": "host cores, rank 0 only"})
-    cpu = {"value": round(value, 3), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-           "sample": f"per step: {sample}, about {per_step:.1f} s"}
+    cores, note = cpu_cores()
+    cpu = {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+           "sample": f"per step: {sample}, about {per_step:.1f} s", "threads_note": note}
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",

@@ -57,7 +57,8 @@ typedef enum {
   DSA_ERR_TIMEOUT = 4,      /* a bounded device wait ran out (see dsa_sync_status)      */
   DSA_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed              */
   DSA_ERR_WORKSPACE = 6,    /* workspace missing or smaller than *_workspace_bytes()    */
-  DSA_ERR_BOUNDS = 7        /* a kernel met an out-of-range index or page and skipped it */
+  DSA_ERR_BOUNDS = 7,       /* a kernel met an out-of-range index or page and skipped it */
+  DSA_ERR_RANGE = 8         /* an input value lies outside the range a kernel supports   */
 } dsa_status;
 
 typedef enum { DSA_BF16 = 0, DSA_E4M3 = 1 } dsa_dtype;
@@ -89,7 +90,9 @@ typedef struct {
  * Index-reuse handle: the Top-k of one Full layer, handed to the Shared layers that
  * follow it and to later MTP draft steps (page sections cited above).
  * idx: caller-owned device buffer [rows, k] int32 (row order within a row unspecified,
- * -1 = padding).  generation is bumped by every call that fills it; filled = 1 after.
+ * -1 = padding).  generation is bumped by every call that fills it; filled = 1 after.  A
+ * filling call sets filled = 0 before it launches anything and back to 1 only once all of
+ * its launches are enqueued, so a fill that fails leaves the handle unfilled.
  */
 typedef struct {
   int32_t* idx;
@@ -177,6 +180,11 @@ dsa_status dsa_topk(const float* scores, int64_t ld, int32_t n_rows, const int32
  *   kv   dim 576.  Dense bf16: idx values are token rows of kv.  Paged e4m3: idx row i is
  *        sequence i and its values are token positions s < seq_lens[i].
  *   A row with no valid index gets out = 0 and lse = -inf.
+ *   Paged e4m3 caches: the products run on f16 operands (e4m3 values are exact in f16), so q is
+ *   converted from bf16 to f16 and must lie within the f16 range, |q| < 65520; a larger value
+ *   would become infinite and is reported as DSA_ERR_RANGE by dsa_sync_status (that row's output
+ *   is then undefined).  Values below 2^-14 keep f16's subnormal precision (absolute error at most
+ *   2^-25).  Dense bf16 caches take any finite bf16 q.
  * workspace: dsa_sparse_mla_workspace_bytes(...) bytes (split-KV partials for few rows).
  */
 size_t dsa_sparse_mla_workspace_bytes(int32_t n_q, int32_t k, const dsa_cache_view* kv);
@@ -278,7 +286,8 @@ int32_t dsa_abi_version(void);
 size_t dsa_abi_sizeof(int32_t which);
 /* Synchronise the stream, then read and clear the device status word of the current
  * device: DSA_ERR_TIMEOUT if a bounded wait ran out, DSA_ERR_BOUNDS if a kernel skipped an
- * out-of-range index/page, DSA_ERR_CUDA on a CUDA error, else DSA_OK. */
+ * out-of-range index/page, DSA_ERR_RANGE if an attention over an e4m3 cache met a query value
+ * outside the f16 range, DSA_ERR_CUDA on a CUDA error, else DSA_OK. */
 dsa_status dsa_sync_status(void* stream);
 /* Test hook: launch one CTA that waits on an mbarrier nothing will complete, bounded by
  * timeout_ns; the kernel then records DSA_ERR_TIMEOUT in the status word and exits. */

@@ -16,9 +16,10 @@ LIB_PATH = os.path.join(HERE, "libdsa.so")
 
 DSA_BF16, DSA_E4M3 = 0, 1
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "stale index handle", 4: "device wait timed out",
-          5: "CUDA error", 6: "workspace too small", 7: "index or page out of range"}
+          5: "CUDA error", 6: "workspace too small", 7: "index or page out of range",
+          8: "input value outside the supported range"}
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_STALE_HANDLE, DSA_ERR_TIMEOUT, DSA_ERR_CUDA, \
-    DSA_ERR_WORKSPACE, DSA_ERR_BOUNDS = range(8)
+    DSA_ERR_WORKSPACE, DSA_ERR_BOUNDS, DSA_ERR_RANGE = range(9)
 
 EXPORTS = [
     "dsa_quant_e4m3", "dsa_indexer_score", "dsa_topk_workspace_bytes", "dsa_topk",

@@ -568,6 +568,7 @@ const char* dsa_status_str(dsa_status s) {
     case DSA_ERR_CUDA: return "CUDA error";
     case DSA_ERR_WORKSPACE: return "workspace too small";
     case DSA_ERR_BOUNDS: return "index or page out of range";
+    case DSA_ERR_RANGE: return "input value outside the supported range";
   }
   return "unknown status";
 }
@@ -599,6 +600,8 @@ dsa_status dsa_sync_status(void* stream) {
   DSA_TRY(cuda_check(cudaMemcpy(ds->status, &zero, sizeof(int), cudaMemcpyHostToDevice), "clear status"));
   if (v & DEVERR_TIMEOUT) return fail(DSA_ERR_TIMEOUT, "a bounded device wait ran out");
   if (v & DEVERR_BOUNDS) return fail(DSA_ERR_BOUNDS, "a kernel skipped an out-of-range index or page");
+  if (v & DEVERR_RANGE)
+    return fail(DSA_ERR_RANGE, "a query value of an attention over an e4m3 cache exceeds the f16 range");
   return DSA_OK;
 }
 
@@ -742,6 +745,10 @@ dsa_status indexshare_group_forward(const dsa_group_args* a, dsa_index_handle* h
                 a->k);
   }
   if (reuse_only && !h->filled) return fail(DSA_ERR_STALE_HANDLE, "reuse of an unfilled index handle");
+  // A fill invalidates the handle before anything can write h->idx; only a fill that enqueues
+  // every one of its launches marks it filled again, so a fill that fails part-way leaves no mix
+  // of old and new indices for a later reuse call to accept.
+  if (!reuse_only) h->filled = 0;
   DeviceState* ds = nullptr;
   DSA_TRY(device_state(&ds));
   GroupPlan g;

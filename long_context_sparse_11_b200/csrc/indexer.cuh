@@ -275,7 +275,9 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
       for (int g = 0; g < C::NGROUP; ++g) {
         if (!group_needed(kt, g)) continue;
         const int bf = job % C::NBUF;
-        if (!mbar_wait(acc_full(bf), (job / C::NBUF) & 1, abort_flag, p.status, p.wait_ns)) {
+        // every lane must take the same branch: the TMEM loads below are warp-collective
+        if (!__all_sync(0xffffffffu, mbar_wait(acc_full(bf), (job / C::NBUF) & 1, abort_flag, p.status,
+                                               p.wait_ns))) {
           ok = false;
           break;
         }

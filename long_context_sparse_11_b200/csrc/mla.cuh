@@ -456,8 +456,10 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
           cp_async16(base + OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7), qsrc + h * 1152 + ch * 16, 16);
         }
       } else {
-        // batches of QB loads in flight before the first conversion
+        // batches of QB loads in flight before the first conversion; values that f16 cannot hold
+        // (|q| >= 65520 rounds to infinity) are reported through the status word
         constexpr int QPER = (QCH + GA_THREADS - 1) / GA_THREADS, QB = 3;  // chunks c >= QCH are skipped
+        bool out_of_range = false;
         for (int b0 = 0; b0 < QPER; b0 += QB) {
           uint4 raw[QB];
 #pragma unroll
@@ -474,12 +476,16 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
             const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
             uint32_t o[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              o[i] = pack_pair(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u), true);
+            for (int i = 0; i < 4; ++i) {
+              const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+              out_of_range |= fmaxf(fabsf(lo), fabsf(hi)) >= 65520.f;
+              o[i] = pack_pair(lo, hi, true);
+            }
             *reinterpret_cast<uint4*>(smem + OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7)) =
                 make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
+        if (out_of_range) atomicOr(p.status, DEVERR_RANGE);
       }
       if (!PAGED) {
         cp_async_arrive_noinc(bar(B_QFULL));
@@ -553,12 +559,18 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
     bool ok = true;
     WorkIter wk = work_begin<SK>(p);
     Item it;
+    // A failed (timed-out) wait is recorded in `fail` and acted on at the next named_bar_or, where
+    // all softmax threads see the same OR and leave together: none is then left waiting at a
+    // later barrier for one that has gone.  Before a warp-collective TMEM access the lanes of a
+    // warp agree on `fail` first (__any_sync).  A failed wait always comes with the CTA's abort
+    // flag set, so the waits that follow it return at once.
     while (ok && work_next<SK>(p, wk, it)) {
       const int32_t seq_len = PAGED ? p.seq_lens[it.irow] : 0;
       const int32_t* idx_row = p.idx + static_cast<int64_t>(it.irow) * p.k;
       if (quad == 0 && head_lane) m_run[hcol + lane] = -INFINITY;
       named_bar(1, SM_THREADS);
-      if (SM_GATHER && it.n_tiles > 0 && !issue(prepare(it, 0, threadIdx.x), gtile)) break;
+      bool fail = false;
+      if (SM_GATHER && it.n_tiles > 0) fail = !issue(prepare(it, 0, threadIdx.x), gtile);
       float lsum[HPW];
 #pragma unroll
       for (int h = 0; h < HPW; ++h) lsum[h] = 0.f;
@@ -571,18 +583,21 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         Plan next_plan;  // indices of the next tile, loaded while this tile's softmax runs
         if (SM_GATHER && t + 1 < it.n_tiles) next_plan = prepare(it, t + 1, threadIdx.x);
         const float kscale = PAGED ? (valid ? p.kv_scale[prow] : 0.f) : 1.f;
-        if (!mbar_wait(bar(B_SFULL), par, abort_flag, p.status, p.wait_ns)) {
-          ok = false;
-          break;
+        {
+          const bool got = mbar_wait(bar(B_SFULL), par, abort_flag, p.status, p.wait_ns);
+          fail = __any_sync(0xffffffffu, fail || !got);   // warp-uniform: the TMEM load is collective
         }
         tc_fence_after();
         float z[HPW];
-        {
+        if (!fail) {
           uint32_t x[HPW];
           tmem_ld_heads<HPW>(tmem + TM_S + 64u * par + hcol + lane_off, x);
           const float zs = p.scale_log2 * kscale;
 #pragma unroll
           for (int h = 0; h < HPW; ++h) z[h] = valid ? __uint_as_float(x[h]) * zs : -INFINITY;
+        } else {
+#pragma unroll
+          for (int h = 0; h < HPW; ++h) z[h] = -INFINITY;
         }
         // Lazy running max: the cross-lane reduction is needed only when some logit exceeds
         // its head's running max by more than 8 (log2 units) -- always on an item's first tile.
@@ -595,7 +610,10 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
                     (z[4 * c + 3] > m4.w + 8.f);
         }
         if (__any_sync(0xffffffffu, exceed) && lane == 0) *need = 1;
-        named_bar(1, SM_THREADS);
+        if (named_bar_or(1, SM_THREADS, fail)) {
+          ok = false;
+          break;
+        }
         if (st == 0) need_flags[(gtile + 1) & 1] = 0;  // the next tile's flag: its readers are done
         const bool resc = *need != 0;
         if (resc) {
@@ -647,13 +665,11 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         }
         if (resc && t > 0) {
           // O^T (dims on lanes, heads on columns) *= alpha; PV of the previous tile is done
-          if (!mbar_wait(bar(B_PVDONE), par ^ 1, abort_flag, p.status, p.wait_ns)) {
-            ok = false;
-            break;
-          }
+          const bool got = mbar_wait(bar(B_PVDONE), par ^ 1, abort_flag, p.status, p.wait_ns);
+          fail = __any_sync(0xffffffffu, fail || !got);
           tc_fence_after();
 #pragma unroll 1
-          for (int mb = 0; mb < 4; ++mb) {
+          for (int mb = 0; mb < 4 && !fail; ++mb) {
             uint32_t x[HPW];
             const uint32_t ta = tmem + 64u * mb + hcol + lane_off;
             tmem_ld_heads<HPW>(ta, x);
@@ -665,22 +681,20 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(bar(B_PFULL));
-        if (SM_GATHER && t + 1 < it.n_tiles && !issue(next_plan, gtile + 1)) {
-          ok = false;
-          break;
-        }
+        if (SM_GATHER && t + 1 < it.n_tiles && !fail) fail = !issue(next_plan, gtile + 1);
       }
       if (!ok) break;
       // ---- end of item: wait for the last PV, reduce row sums, write the output
       if (it.n_tiles > 0) {
-        if (!mbar_wait(bar(B_PVDONE), (gtile - 1) & 1, abort_flag, p.status, p.wait_ns)) break;
+        const bool got = mbar_wait(bar(B_PVDONE), (gtile - 1) & 1, abort_flag, p.status, p.wait_ns);
+        fail = __any_sync(0xffffffffu, fail || !got);
         tc_fence_after();
       }
       {
         const float wsum = warp_reduce_heads<false, HPW>(lsum, lane);
         if (reduce_lane_writes<HPW>(lane)) red[quad * 64 + hcol + reduce_head_of_lane<HPW>(lane)] = wsum;
       }
-      named_bar(1, SM_THREADS);
+      if (named_bar_or(1, SM_THREADS, fail)) break;
       if (quad == 0 && head_lane) {
         const int h = hcol + lane;
         l_tot[h] = red[h] + red[64 + h] + red[128 + h] + red[192 + h];

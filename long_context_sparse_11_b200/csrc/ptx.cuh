@@ -8,7 +8,7 @@
 namespace dsa {
 
 // Device-side status word bits (read back by dsa_sync_status).
-enum : int { DEVERR_TIMEOUT = 1, DEVERR_BOUNDS = 2 };
+enum : int { DEVERR_TIMEOUT = 1, DEVERR_BOUNDS = 2, DEVERR_RANGE = 4 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -68,6 +68,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 
 __device__ __forceinline__ void named_bar(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Named barrier that also ORs one predicate over the participating threads: every thread gets
+// the same result, so a group of warps can agree to leave a loop together (no thread is left
+// waiting at a later barrier for one that has gone).
+__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbarrier.cta.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA / tcgen05.mma).
 __device__ __forceinline__ void fence_async_smem() {

@@ -34,7 +34,7 @@ from .generators import (
 )
 
 __all__ = ["PrefillSpec", "DecodeSpec", "WORKLOADS", "make_prefill", "make_decode",
-           "decode_context_lengths", "page_table", "make_decode_indexer",
+           "decode_context_lengths", "page_table", "make_decode_indexer", "make_decode_new_tokens",
            "IDX_HEADS", "IDX_DIM", "MLA_HEADS", "D_QK", "D_V", "PAGE"]
 
 IDX_HEADS, IDX_DIM = 32, 128
@@ -43,6 +43,7 @@ PAGE = 64
 
 T_QIDX, T_W, T_KIDX, T_Q, T_KV, T_PERM, T_CTX, T_KSCALE, T_KVSCALE = range(1, 10)
 T_QIDX_DRAFT, T_W_DRAFT = 10, 11   # indexer query and weights of draft rows (per-row Top-k only)
+T_NEW_KV, T_NEW_KEY = 12, 13         # a decode step's new token rows (latent row, indexer key)
 
 
 @dataclass
@@ -210,6 +211,18 @@ def make_decode_indexer(spec: DecodeSpec, layer: int, n_pages: int, batch: int, 
     keys, sc = _fp8_pool(sub_seed(s, layer, T_KIDX), n_pages, IDX_DIM, device)
     return {"q_idx": _bf16(q, device).reshape(batch, IDX_HEADS, IDX_DIM), "w": w, "idx_keys": keys,
             "idx_key_scale": sc}
+
+
+def make_decode_new_tokens(spec: DecodeSpec, batch: int, layers, full_layers, device=None) -> dict:
+    """The rows a decode step appends for its current token (position N_b - 1 of each sequence):
+    a latent row [B,576] bf16 ~N(0,1) for every layer in ``layers`` and an indexer key row
+    [B,128] bf16 ~N(0,1) for every Full layer in ``full_layers`` (streams keyed by the layer)."""
+    s = spec.seed
+    kv = {l: _bf16(_normal(sub_seed(s, l, T_NEW_KV), batch * D_QK, device), device).reshape(batch, D_QK)
+          for l in layers}
+    key = {l: _bf16(_normal(sub_seed(s, l, T_NEW_KEY), batch * IDX_DIM, device), device).reshape(batch, IDX_DIM)
+           for l in full_layers}
+    return {"kv": kv, "key": key}
 
 
 def make_decode(spec: DecodeSpec, device=None, ctx=None, layers=None) -> dict:

@@ -53,8 +53,8 @@ def test_schedule_agrees_with_oracle(lib):
 
 
 def test_status_strings(lib):
-    for s in range(8):
-        assert lib.dsa_status_str(s)
+    for s in range(9):
+        assert lib.dsa_status_str(s).decode() != "unknown status"
 
 
 def _err(lib):
@@ -151,6 +151,15 @@ def test_group_handle_checks(lib):
     h = B.IndexHandle(256, 100, 64, 0, -1, 0)
     assert lib.indexshare_group_forward(ctypes.byref(a), ctypes.byref(h), 1, None) == B.DSA_ERR_STALE_HANDLE
     assert "unfilled" in _err(lib)
+    # a fill that fails leaves the handle unfilled, so a reuse call cannot accept indices that the
+    # failed fill may have half overwritten.  No workspace is given: the fill fails before any
+    # launch, for want of a device here or of the workspace on a GPU machine.
+    assert a.workspace is None and a.workspace_bytes == 0
+    h = B.IndexHandle(256, 100, 64, 1, 0, 3)
+    rc = lib.indexshare_group_forward(ctypes.byref(a), ctypes.byref(h), 0, None)
+    assert rc in (B.DSA_ERR_CUDA, B.DSA_ERR_WORKSPACE)
+    assert h.filled == 0 and h.generation == 3
+    assert lib.indexshare_group_forward(ctypes.byref(a), ctypes.byref(h), 1, None) == B.DSA_ERR_STALE_HANDLE
     # too many layers
     a.n_layers = 5
     assert lib.indexshare_group_forward(ctypes.byref(a), ctypes.byref(h), 0, None) == B.DSA_ERR_INVALID_ARG

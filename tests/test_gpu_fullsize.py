@@ -4,6 +4,7 @@ rows that the fp64 oracle computes one by one (needs a B200).
 * prefill_32k       L=32,768, Top-2048, bf16 indexer with AR(1) keys, 4 layers
 * prefill_128k_fp8  L=131,072, Top-2048, FP8 indexer quantised on the path, 4 layers
 * decode_b32_mtp4   32 sequences of 65K..262K tokens, 5 rows each, paged FP8 caches
+* decode_1m_mtp5    1 sequence of 1,048,576 tokens, 6 rows, the 78-layer schedule (21 groups)
 Tolerances as in test_gpu_kernels.py / test_gpu_group.py.
 """
 import math
@@ -133,3 +134,59 @@ def test_fullsize_decode_b32_mtp4():
                 ref, _ = O.sparse_mla_row(O.bf16_to_f64(Q[row]), rows_kv, np.arange(len(sel)), spec.softmax_scale)
                 ma, rl = attn_errors(o[row], ref)
                 assert ma <= 2e-2 and rl <= 5e-3, (l, row, ma, rl)
+
+
+def test_fullsize_decode_1m_mtp5_78_layer_schedule():
+    """decode_1m_mtp5: one sequence of 1,048,576 tokens, 1 + 5 rows, the 78-layer schedule run as
+    21 IndexShare groups exactly as the benchmark runs them.  Checked: each group's handle comes
+    from its own Full layer; the Top-k sets of Full layers 0, 2 and 74 against the oracle on the
+    path's e4m3 keys; and all 6 rows of layers 0, 1, 5 and 77 (Full, Full, Shared of 2, Shared of
+    74) against the oracle on the GPU's indices."""
+    from synth import make_decode_indexer
+    spec = WORKLOADS["decode_1m_mtp5"]
+    inp = make_decode(spec, device="cuda")
+    n, R = int(inp["ctx"][0]), spec.rows_per_seq
+    ctx_d = torch.from_numpy(inp["ctx"].astype(np.int32)).cuda()
+    bt_d = torch.from_numpy(inp["block_table"]).cuda()
+    kvs = [dsa.paged_view(inp["KV"][l], inp["KV_scale"][l], bt_d, ctx_d) for l in range(spec.n_layers)]
+    fulls = [l for l in range(spec.n_layers) if dsa.layer_is_full(l)]
+    assert len(fulls) == 21
+    groups, indexers = {}, {}
+    for f, e in zip(fulls, fulls[1:] + [spec.n_layers]):
+        ind = inp if f == 0 else make_decode_indexer(spec, f, inp["n_pages"], 1, "cuda")
+        keys = dsa.paged_view(ind["idx_keys"], ind["idx_key_scale"], bt_d, ctx_d)
+        g = dsa.IndexShareGroup(ind["q_idx"], ind["w"], keys, spec.k, inp["Q"][f:e], kvs[f:e], inp["softmax_scale"],
+                                indexer_dtype=dsa.DSA_E4M3, q_rows_per_idx_row=R, first_layer=f)
+        g.forward()
+        groups[f] = g
+        if f in (0, 2, 74):
+            indexers[f] = ind
+    dsa.sync_status()
+    for f, g in groups.items():
+        assert g.handle.filled == 1 and g.handle.producer_layer == f and g.handle.generation == 1
+    bt = inp["block_table"]
+    for f, ind in indexers.items():
+        q8, sq = O.quantize_e4m3_rows(host_bits(ind["q_idx"]), 128)
+        qv = O.e4m3_to_f64(q8) * sq.reshape(-1, 32, 1)
+        kk = O.paged_rows(ind["idx_keys"].cpu().numpy(), ind["idx_key_scale"].cpu().numpy(), bt[0], n)
+        sc = O.indexer_scores(qv, ind["w"].cpu().numpy().astype(np.float64), kk, [n])[0]
+        check_topk_sets(groups[f].idx[0].cpu().numpy(), sc, n, spec.k)
+        del kk, sc
+    for l in (0, 1, 5, 77):
+        f = dsa.layer_producer(l)
+        idx = groups[f].idx[0].cpu().numpy()
+        sel = idx[idx >= 0]
+        pages, slots = bt[0][sel // 64], sel % 64
+        kvp = inp["KV"][l][torch.from_numpy(pages.astype(np.int64)).cuda(),
+                           torch.from_numpy(slots.astype(np.int64)).cuda()].cpu().numpy()
+        kvs_ = inp["KV_scale"][l][torch.from_numpy(pages.astype(np.int64)).cuda(),
+                                  torch.from_numpy(slots.astype(np.int64)).cuda()].cpu().numpy()
+        rows_kv = O.e4m3_to_f64(kvp) * kvs_.astype(np.float64)[:, None]
+        o = O.bf16_to_f64(host_bits(groups[f].out[l - f]))
+        Q = host_bits(inp["Q"][l])
+        for r in range(R):
+            ref, _ = O.sparse_mla_row(O.bf16_to_f64(Q[r]), rows_kv, np.arange(len(sel)), spec.softmax_scale)
+            ma, rl = attn_errors(o[r], ref)
+            assert ma <= 2e-2 and rl <= 5e-3, (l, r, ma, rl)
+    del groups, inp, kvs
+    torch.cuda.empty_cache()

@@ -21,6 +21,7 @@ pytestmark = pytest.mark.gpu
 import long_context_sparse_11_b200 as dsa  # noqa: E402
 import oracle.dsa_oracle as O  # noqa: E402
 from synth import make_prefill, make_decode, PrefillSpec, DecodeSpec, WORKLOADS  # noqa: E402
+from synth.generators import bf16_bits_np  # noqa: E402
 from test_gpu_kernels import (bf16_dev, u8_dev, f32_dev, i32_dev, bf16_host, check_topk_sets,  # noqa: E402
                               attn_errors)
 
@@ -225,3 +226,76 @@ def test_decode_group_replays_from_a_captured_cuda_graph():
     for a, b in zip(got[2:], g.lse):
         assert torch.max(torch.abs(a - b)).item() <= 1e-3
     del graph
+
+
+def _paged_group(spec, inp, rows_per_view=1):
+    ctx_d, bt_d = i32_dev(inp["ctx"]), i32_dev(inp["block_table"])
+    keys = dsa.paged_view(u8_dev(inp["idx_keys"]), f32_dev(inp["idx_key_scale"]), bt_d, ctx_d)
+    kvs = [dsa.paged_view(u8_dev(inp["KV"][l]), f32_dev(inp["KV_scale"][l]), bt_d, ctx_d)
+           for l in range(spec.n_layers)]
+    q_idx, w, Q = bf16_dev(inp["q_idx"]), f32_dev(inp["w"]), [bf16_dev(x) for x in inp["Q"]]
+    g = dsa.IndexShareGroup(q_idx, w, keys, spec.k, Q, kvs, inp["softmax_scale"], indexer_dtype=dsa.DSA_E4M3,
+                            q_rows_per_idx_row=spec.rows_per_seq)
+    return g, q_idx, Q
+
+
+def test_decode_draft_step_reuses_the_handle():
+    """MTP draft steps >= 2: a reuse_only call with new query rows (and a changed indexer query,
+    which it must not read) keeps the handle's indices and generation and attends with them."""
+    spec = DecodeSpec("r", batch=4, ctx_lo=300, ctx_hi=9000, rows_per_seq=3, k=256, n_layers=2, seed=11)
+    inp = make_decode(spec)
+    g, q_idx, Q = _paged_group(spec, inp)
+    g.forward()
+    dsa.sync_status()
+    idx0, gen0 = g.idx.clone(), g.handle.generation
+    assert g.handle.filled == 1 and gen0 == 1
+    rng = np.random.default_rng(2)
+    new_q = [bf16_bits_np(rng.normal(size=x.shape)) for x in inp["Q"]]
+    for dst, src in zip(Q, new_q):
+        dst.copy_(bf16_dev(src))
+    q_idx.copy_(bf16_dev(bf16_bits_np(rng.normal(size=inp["q_idx"].shape))))
+    out, lse = g.forward(reuse_only=True)
+    dsa.sync_status()
+    assert torch.equal(g.idx, idx0) and g.handle.generation == gen0
+    idx = idx0.cpu().numpy()
+    R = spec.rows_per_seq
+    for l in range(2):
+        o, ls = O.bf16_to_f64(bf16_host(out[l])), lse[l].cpu().numpy()
+        for b in range(spec.batch):
+            kv = O.paged_rows(inp["KV"][l], inp["KV_scale"][l], inp["block_table"][b], int(inp["ctx"][b]))
+            for r in range(R):
+                row = b * R + r
+                ref, ref_lse = O.sparse_mla_row(O.bf16_to_f64(new_q[l][row]), kv, idx[b], inp["softmax_scale"])
+                ma, rel = attn_errors(o[row], ref)
+                assert ma <= 2e-2 and rel <= 5e-3, (l, row, ma, rel)
+                assert np.max(np.abs(ls[row] - ref_lse)) <= 2e-3
+
+
+def test_paged_attention_query_values_within_and_beyond_f16_range():
+    """Attention over an e4m3 cache runs its products on f16 operands: query values up to the f16
+    range give the oracle's result; a value beyond it is reported as DSA_ERR_RANGE."""
+    spec = DecodeSpec("q", batch=3, ctx_lo=200, ctx_hi=3000, rows_per_seq=2, k=128, n_layers=1, seed=13)
+    inp = make_decode(spec)
+    Qb = O.bf16_to_f64(inp["Q"][0]).copy()
+    Qb[:, 0, :4] = [20000.0, -20000.0, 12288.0, -30720.0]      # large, still finite in f16
+    Qb[:, 5, 100] = 65280.0                                     # the largest bf16 value f16 holds
+    inp["Q"][0] = bf16_bits_np(Qb)
+    Qb = O.bf16_to_f64(inp["Q"][0]).copy()                      # the values as rounded to bf16
+    g, _, Q = _paged_group(spec, inp)
+    out, lse = g.forward()
+    dsa.sync_status()
+    idx, o = g.idx.cpu().numpy(), O.bf16_to_f64(bf16_host(out[0]))
+    for b in range(spec.batch):
+        kv = O.paged_rows(inp["KV"][0], inp["KV_scale"][0], inp["block_table"][b], int(inp["ctx"][b]))
+        for r in range(spec.rows_per_seq):
+            row = b * spec.rows_per_seq + r
+            ref, _ = O.sparse_mla_row(Qb[row], kv, idx[b], inp["softmax_scale"])
+            ma, rel = attn_errors(o[row], ref)
+            assert ma <= 2e-2 and rel <= 5e-3, (row, ma, rel)
+    Qb[1, 7, 9] = 1.0e5                                         # beyond f16
+    Q[0].copy_(bf16_dev(bf16_bits_np(Qb)))
+    g.forward(reuse_only=True)
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.sync_status()
+    assert e.value.status == dsa.binding.DSA_ERR_RANGE
+    dsa.sync_status()                                           # the status word was cleared
