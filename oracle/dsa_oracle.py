@@ -51,6 +51,16 @@ R10 The paged FP8 latent cache holds all 576 dims as e4m3 with one fp32 scale pe
     (the pages name an FP8 KV cache, [forum] "vLLM推理启动", but not its layout).
 R11 Paged caches: token s of sequence b sits in page block_table[b][s // 64], slot s % 64
     (the pages give no block size).
+R12 Indexer inputs (what feeds R1): q_idx[t] = cq[t] Wq^T split into 32 heads of 128, from the
+    query latent cq of rank 2,048; k[t] = LayerNorm(x[t] Wk^T) * gamma + beta over the 128 key
+    dims (eps 1e-6, biased variance), and w[t] = x[t] Ww^T, from the hidden state x of width
+    6,144 ([ailearn] "一枚 Token，怎样穿过 78 层": hidden 6,144, 32 indexer heads; "IndexShare：
+    四层共用一次搜索结果": 9,371,904 parameters per indexer, which these shapes reproduce).  No
+    rotary embedding inside the indexer (the pages give none).
+R13 Latent KV rows (what feeds R4): row[t] = [RMSNorm(x[t] W_dkv^T) * gamma (512 dims, eps 1e-6) ||
+    RoPE(x[t] W_kr^T, t) (64 dims)]; the query's 64 RoPE dims are rotated the same way at their
+    own position ([ailearn] architecture card: KV joint compression of rank 512, RoPE theta
+    8,000,000 over 2^20 positions).  RoPE turns pair (2i, 2i+1) by the angle pos * theta^(-2i/64).
 """
 from __future__ import annotations
 
@@ -62,13 +72,16 @@ __all__ = [
     "bf16_to_f64", "e4m3_to_f64", "quantize_e4m3_rows", "cache_write_e4m3", "indexer_scores",
     "topk_row", "sparse_mla_row", "dense_causal_attention_row", "prefill_tables",
     "group_prefill", "paged_rows", "group_decode", "group_decode_per_row", "layer_schedule", "indexer_param_count",
-    "E4M3_MAX", "IDX_HEADS", "IDX_DIM", "MLA_HEADS", "D_QK", "D_V", "PAGE",
+    "E4M3_MAX", "IDX_HEADS", "IDX_DIM", "MLA_HEADS", "D_QK", "D_V", "PAGE", "ROPE_THETA", "NORM_EPS",
+    "layer_norm", "rms_norm", "rope_pairs", "indexer_projections", "mla_latent_rows", "rope_query",
 ]
 
 E4M3_MAX = 448.0
 IDX_HEADS, IDX_DIM = 32, 128        # [ailearn] architecture card: 32 indexer heads
 MLA_HEADS, D_QK, D_V = 64, 576, 512  # [ailearn] architecture card: 64 heads, KV rank 512 (+64 RoPE, R4)
 PAGE = 64
+ROPE_THETA = 8.0e6                    # [ailearn] architecture card
+NORM_EPS = 1e-6                       # R12, R13
 
 
 # ----------------------------------------------------------------------------- number formats
@@ -374,3 +387,62 @@ def indexer_param_count(q_rank: int = 2048, hidden: int = 6144, heads: int = IDX
     hidden size 6,144 and the 32 heads are on [ailearn] ("一枚 Token，怎样穿过 78 层");
     the 2,048 query rank and the LayerNorm are this file's reading.  Check only."""
     return q_rank * heads * dim + hidden * dim + hidden * heads + 2 * dim
+
+
+# ----------------------------------------------------------------------------- inputs of the path
+
+
+def layer_norm(x, gamma, beta, eps: float = NORM_EPS) -> np.ndarray:
+    """Per-row LayerNorm over the last axis (R12): (x - mean) / sqrt(var + eps) * gamma + beta,
+    var the biased (1/n) variance."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * np.asarray(gamma, dtype=np.float64) + np.asarray(beta, dtype=np.float64)
+
+
+def rms_norm(x, gamma, eps: float = NORM_EPS) -> np.ndarray:
+    """Per-row RMSNorm over the last axis (R13): x / sqrt(mean(x^2) + eps) * gamma."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt((x ** 2).mean(axis=-1, keepdims=True) + eps) * np.asarray(gamma, dtype=np.float64)
+
+
+def rope_pairs(x, pos, theta: float = ROPE_THETA) -> np.ndarray:
+    """Rotary embedding of the last axis (64 dims, R13): pair (2i, 2i+1) of a vector at position
+    pos turns by the angle pos * theta^(-2i/64)."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    freq = theta ** (-np.arange(0, d, 2, dtype=np.float64) / d)          # [d/2]
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * freq             # [..., d/2]
+    c, s = np.cos(ang), np.sin(ang)
+    out = np.empty_like(x)
+    out[..., 0::2] = x[..., 0::2] * c - x[..., 1::2] * s
+    out[..., 1::2] = x[..., 0::2] * s + x[..., 1::2] * c
+    return out
+
+
+def indexer_projections(cq, x, Wq, Wk, Ww, gamma, beta):
+    """Indexer inputs of T tokens (R12): cq [T,2048], x [T,6144] values; Wq [4096,2048],
+    Wk [128,6144], Ww [32,6144] (output x input); gamma, beta [128].
+    Returns q_idx [T,32,128], k [T,128], w [T,32] in fp64."""
+    cq, x = np.asarray(cq, dtype=np.float64), np.asarray(x, dtype=np.float64)
+    q = cq @ np.asarray(Wq, dtype=np.float64).T
+    k = layer_norm(x @ np.asarray(Wk, dtype=np.float64).T, gamma, beta)
+    w = x @ np.asarray(Ww, dtype=np.float64).T
+    return q.reshape(len(q), IDX_HEADS, IDX_DIM), k, w
+
+
+def mla_latent_rows(x, W_dkv, W_kr, gamma, pos):
+    """Latent KV rows of T tokens (R13): x [T,6144]; W_dkv [512,6144], W_kr [64,6144]; gamma [512];
+    pos [T].  Returns [T,576] = [RMSNorm(x W_dkv^T) * gamma || RoPE(x W_kr^T, pos)] in fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    c = rms_norm(x @ np.asarray(W_dkv, dtype=np.float64).T, gamma)
+    r = rope_pairs(x @ np.asarray(W_kr, dtype=np.float64).T, pos)
+    return np.concatenate([c, r], axis=-1)
+
+
+def rope_query(q, pos) -> np.ndarray:
+    """The query side of R13: q [T,64,576] with dims 512..575 of every head turned to position pos[t]."""
+    q = np.array(q, dtype=np.float64, copy=True)
+    q[:, :, D_V:] = rope_pairs(q[:, :, D_V:], np.asarray(pos)[:, None])
+    return q

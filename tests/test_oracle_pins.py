@@ -549,3 +549,129 @@ def _mutant_src(fn, edits):
     ns = dict(vars(O))
     exec(compile(src, "<mutant>", "exec"), ns)
     return ns[fn.__name__]
+
+
+# ----------------------------------------------------------------------------- inputs of the path (R12, R13)
+
+
+def test_layer_norm_closed_forms(fn=None):
+    fn = fn or O.layer_norm
+    x = np.array([[1.0, 3.0] * 64, [5.0] * 128, [-2.0, 0.0, 2.0, 0.0] * 32])
+    g, b = np.full(128, 2.0), np.full(128, 0.5)
+    y = fn(x, g, b)
+    # row 0: mean 2, biased variance 1 -> +-1 / sqrt(1 + eps) ; row 1: constant -> beta
+    assert np.allclose(y[0, :2], [0.5 - 2 / math.sqrt(1 + 1e-6), 0.5 + 2 / math.sqrt(1 + 1e-6)], atol=1e-12)
+    assert np.allclose(y[1], 0.5, atol=1e-12)
+    # row 2: mean 0, variance 2 -> values / sqrt(2 + eps)
+    assert np.allclose(y[2, :3], 0.5 + 2 * np.array([-2.0, 0.0, 2.0]) / math.sqrt(2 + 1e-6), atol=1e-12)
+    z = fn(np.random.default_rng(1).normal(3, 5, size=(4, 128)), np.ones(128), np.zeros(128))
+    assert np.allclose(z.mean(axis=1), 0, atol=1e-12) and np.allclose((z ** 2).mean(axis=1), 1, atol=1e-5)
+
+
+def test_rms_norm_closed_forms(fn=None):
+    fn = fn or O.rms_norm
+    g = np.linspace(0.5, 1.5, 512)
+    x = np.full((1, 512), -3.0)
+    assert np.allclose(fn(x, g), -3.0 / math.sqrt(9.0 + 1e-6) * g, atol=1e-12)
+    r = np.random.default_rng(2).normal(size=(3, 512))
+    assert np.allclose(fn(r, np.ones(512)), fn(1000.0 * r, np.ones(512)), atol=1e-6)   # scale invariant
+    assert np.allclose((fn(r, np.ones(512)) ** 2).mean(axis=1), 1.0, atol=1e-5)
+
+
+def test_rope_closed_forms(fn=None):
+    fn = fn or O.rope_pairs
+    d, th = 64, 8.0e6
+    for i in (0, 1, 17, 31):
+        for p in (0, 1, 1000, (1 << 20) - 1):
+            e = np.zeros(d)
+            e[2 * i] = 1.0
+            y = fn(e, p, th)
+            a = p * th ** (-2 * i / d)
+            assert abs(y[2 * i] - math.cos(a)) < 1e-12 and abs(y[2 * i + 1] - math.sin(a)) < 1e-12
+            assert np.count_nonzero(np.abs(y) > 1e-15) <= 2
+    v = np.random.default_rng(3).normal(size=(5, d))
+    assert np.array_equal(fn(v, np.zeros(5), th), v)                              # position 0: no turn
+    assert np.allclose(np.linalg.norm(fn(v, np.arange(5) * 7.0, th), axis=1), np.linalg.norm(v, axis=1))
+    # relative position: <R(a, m), R(b, n)> depends on m - n only
+    a_, b_ = v[0], v[1]
+    s1 = fn(a_, 100.0, th) @ fn(b_, 37.0, th)
+    s2 = fn(a_, 5100.0, th) @ fn(b_, 5037.0, th)
+    assert abs(s1 - s2) < 1e-9
+
+
+def test_indexer_projections_closed_forms_and_param_count(fn=None):
+    fn = fn or O.indexer_projections
+    rng = np.random.default_rng(4)
+    T = 3
+    cq, x = rng.normal(size=(T, 2048)), rng.normal(size=(T, 6144))
+    Wq = np.zeros((4096, 2048))
+    Wq[np.arange(2048), np.arange(2048)] = 1.0                 # heads 0..15 copy cq, heads 16..31 are 0
+    Wk = np.zeros((128, 6144))
+    Wk[np.arange(128), 6000 + np.arange(128) % 100] = 1.0      # key dim j reads hidden dim 6000 + j % 100
+    Ww = np.zeros((32, 6144))
+    Ww[np.arange(32), 3 * np.arange(32)] = 2.0
+    g, b = np.full(128, 1.5), np.full(128, -0.25)
+    q, k, w = fn(cq, x, Wq, Wk, Ww, g, b)
+    assert q.shape == (T, 32, 128) and k.shape == (T, 128) and w.shape == (T, 32)
+    assert np.array_equal(q[:, :16].reshape(T, 2048), cq) and (q[:, 16:] == 0).all()
+    kk = x[:, 6000 + np.arange(128) % 100]
+    mu, var = kk.mean(axis=1, keepdims=True), kk.var(axis=1, keepdims=True)
+    assert np.allclose(k, (kk - mu) / np.sqrt(var + 1e-6) * 1.5 - 0.25, atol=1e-12)
+    assert np.array_equal(w, 2.0 * x[:, 3 * np.arange(32)])
+    assert Wq.size + Wk.size + Ww.size + g.size + b.size == O.indexer_param_count() == GOLD["params_per_indexer"]["value"]
+
+
+def test_mla_latent_rows_closed_forms(fn=None):
+    fn = fn or O.mla_latent_rows
+    rng = np.random.default_rng(5)
+    x = rng.normal(size=(4, 6144))
+    Wd = np.zeros((512, 6144))
+    Wd[np.arange(512), np.arange(512)] = 1.0
+    Wr = np.zeros((64, 6144))
+    Wr[np.arange(64), 1000 + np.arange(64)] = 1.0
+    g = np.linspace(0.9, 1.1, 512)
+    pos = np.array([0, 1, 77, (1 << 20) - 1])
+    y = fn(x, Wd, Wr, g, pos)
+    assert y.shape == (4, 576)
+    c = x[:, :512]
+    assert np.allclose(y[:, :512], c / np.sqrt((c ** 2).mean(axis=1, keepdims=True) + 1e-6) * g, atol=1e-12)
+    assert np.array_equal(y[0, 512:], x[0, 1000:1064])                            # position 0: not turned
+    for t in range(1, 4):
+        for i in (0, 9, 31):
+            a = pos[t] * 8.0e6 ** (-2 * i / 64)
+            u, v = x[t, 1000 + 2 * i], x[t, 1001 + 2 * i]
+            assert abs(y[t, 512 + 2 * i] - (u * math.cos(a) - v * math.sin(a))) < 1e-9
+            assert abs(y[t, 513 + 2 * i] - (u * math.sin(a) + v * math.cos(a))) < 1e-9
+
+
+def test_rope_query_turns_only_the_rope_dims():
+    rng = np.random.default_rng(6)
+    q = rng.normal(size=(2, 64, 576))
+    y = O.rope_query(q, np.array([0, 500]))
+    assert np.array_equal(y[:, :, :512], q[:, :, :512]) and np.array_equal(y[0], q[0])
+    assert np.allclose(y[1, 7, 512:], O.rope_pairs(q[1, 7, 512:], 500))
+    # a query and a latent key turned to their positions: the RoPE logit depends on their distance
+    kr = rng.normal(size=64)
+    s1 = O.rope_query(q[:1], np.array([900]))[0, 3, 512:] @ O.rope_pairs(kr, 400)
+    s2 = O.rope_query(q[:1], np.array([1500]))[0, 3, 512:] @ O.rope_pairs(kr, 1000)
+    assert abs(s1 - s2) < 1e-9
+
+
+@pytest.mark.parametrize("fn,test,old,new", [
+    ("layer_norm", "test_layer_norm_closed_forms", "var + eps", "var"),                  # eps dropped
+    ("layer_norm", "test_layer_norm_closed_forms", "mean(axis=-1, keepdims=True)\n", "mean()\n"),  # over the tensor
+    ("rms_norm", "test_rms_norm_closed_forms", "(x ** 2).mean(", "np.abs(x).mean("),      # mean |x| for rms
+    ("rope_pairs", "test_rope_closed_forms", "out[..., 1::2] = x[..., 0::2] * s + x[..., 1::2] * c",
+     "out[..., 1::2] = -x[..., 0::2] * s + x[..., 1::2] * c"),                            # turned the wrong way
+    ("rope_pairs", "test_rope_closed_forms", "np.arange(0, d, 2, dtype=np.float64) / d",
+     "np.arange(0, d // 2, dtype=np.float64) / d"),                                       # theta^(-i/64)
+    ("indexer_projections", "test_indexer_projections_closed_forms_and_param_count",
+     "layer_norm(x @ np.asarray(Wk, dtype=np.float64).T, gamma, beta)",
+     "layer_norm(x @ np.asarray(Wk, dtype=np.float64).T, beta, gamma)"),                  # affine swapped
+    ("mla_latent_rows", "test_mla_latent_rows_closed_forms", "rope_pairs(x @ np.asarray(W_kr, dtype=np.float64).T, pos)",
+     "rope_pairs(x @ np.asarray(W_kr, dtype=np.float64).T, pos + 1)"),                    # position off by one
+])
+def test_planted_input_path_mistakes_are_caught(fn, test, old, new):
+    bad = _mutant(getattr(O, fn), old, new)
+    with pytest.raises(AssertionError):
+        globals()[test](bad)
