@@ -269,6 +269,71 @@ dsa_status dsa_topk_no_alloc(const float* scores, int64_t ld, int32_t n_rows, co
                              int64_t causal_len0, int64_t max_len, int32_t k, int32_t* idx_out, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * The inputs of the indexer (the step before a2): its query from the query latent, its key and
+ * per-head weights from the hidden state (ailearn "一枚 Token，怎样穿过 78 层": hidden size 6,144,
+ * 32 indexer heads of 128; "IndexShare：四层共用一次搜索结果": 9,371,904 parameters per indexer,
+ * which the shapes below reproduce with q_rank = 2,048 and hidden = 6,144; the LayerNorm on the
+ * key and the rank of the query latent are this library's reading):
+ *   q_out[t]  = cq[t] . Wq^T                             [T, 4096] = [T, 32, 128] bf16
+ *   k_out[t]  = LayerNorm(x[t] . Wk^T) * gamma + beta    [T, 128] bf16 (eps 1e-6, biased variance)
+ *   w_out[t]  = x[t] . Ww^T                              [T, 32] fp32
+ *   cq   [T, q_rank] bf16;  x [T, hidden] bf16;  Wq [4096, q_rank] bf16 (row = output);
+ *   Wkw  [160, hidden] bf16: rows 0..127 = Wk, rows 128..159 = Ww;  gamma, beta [128] fp32.
+ *   q_rank and hidden: positive multiples of 64.  Products on the tensor cores (bf16 in, fp32
+ *   accumulate).  workspace: dsa_indexer_project_workspace_bytes(T) bytes of device memory.
+ */
+size_t dsa_indexer_project_workspace_bytes(int32_t n_tokens);
+dsa_status dsa_indexer_project(const void* cq, const void* x, const void* Wq, const void* Wkw, const float* gamma,
+                               const float* beta, int32_t n_tokens, int32_t q_rank, int32_t hidden, void* q_out,
+                               void* k_out, float* w_out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * The latent KV rows that sparse MLA reads (ailearn architecture card: KV joint compression of
+ * rank 512, RoPE with theta = 8,000,000 over 2^20 positions; the RMSNorm, the 64 RoPE dims and
+ * the pairing of the rotation are this library's reading):
+ *   latent_out[t] = [ RMSNorm(x[t] . W_dkv^T) * gamma  ||  RoPE(x[t] . W_kr^T, pos[t]) ]   [T, 576] bf16
+ *   RMSNorm: v / sqrt(mean(v^2) + 1e-6).  RoPE: pair (2i, 2i + 1) of the 64 dims turned by the
+ *   angle pos * theta^(-2i/64) (the angle is reduced in double precision).
+ *   x [T, hidden] bf16;  Wkv [576, hidden] bf16: rows 0..511 = W_dkv, rows 512..575 = W_kr;
+ *   gamma [512] fp32;  pos [T] int32 (>= 0).  workspace: dsa_mla_latent_workspace_bytes(T).
+ * dsa_rope_query turns dims 512..575 of every head of q [T, 64, 576] bf16 in place, the same way,
+ * to position pos[t], so that the RoPE part of a logit depends on the distance of the two tokens.
+ */
+size_t dsa_mla_latent_workspace_bytes(int32_t n_tokens);
+dsa_status dsa_mla_latent(const void* x, const void* Wkv, const float* gamma, const int32_t* pos, int32_t n_tokens,
+                          int32_t hidden, float theta, void* latent_out, void* workspace, size_t workspace_bytes,
+                          void* stream);
+dsa_status dsa_rope_query(void* q, const int32_t* pos, int32_t n_q, float theta, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Split-N decode of one long sequence over G GPUs (the pages' full 1M context starts at 8 B200s
+ * with an FP8 KV cache, ailearn deployment section "CP · EP · P/D · HiCache"; the split itself is
+ * this library's design).  Rank r holds the contiguous cache slice of positions [lo_r, hi_r) and
+ * runs a2-a4 on it (dsa_indexer_score / dsa_topk over the slice, local positions); then:
+ *   dsa_split_candidates: local Top-k idx_local [n_rows, k] of the slice's scores
+ *     [n_rows, ld] -> cand_score / cand_idx [n_rows, k]: (score, lo_r + position) ordered by
+ *     position, padding (-inf, -1) last.  Positions >= n_local are skipped (DSA_ERR_BOUNDS).
+ *   (the caller gathers every rank's candidates, in rank order, into [n_rows, G * k])
+ *   dsa_split_merge: the k best of the n_cand = G * k candidates of each row -> idx_global
+ *     [n_rows, k] (the same on every rank, equal to the Top-k of the unsplit row: equal scores go
+ *     to the lower position) and idx_local [n_rows, k] = idx_global - lo for positions in
+ *     [lo, hi), else -1, for dsa_sparse_mla_attn over this rank's slice (with lse).
+ *     n_cand a multiple of 4; workspace: dsa_split_merge_workspace_bytes(...).
+ *   (the caller gathers every rank's out / lse into o_parts [G, n_q, 64, 512] bf16 and
+ *   lse_parts [G, n_q, 64] fp32)
+ *   dsa_combine_partials: lse = log sum_r exp(lse_r), out = sum_r exp(lse_r - lse) out_r
+ *     [n_q, 64, 512] bf16; lse may be NULL.  A part with lse_r = -inf contributes nothing.
+ */
+dsa_status dsa_split_candidates(const float* scores, int64_t ld, int32_t n_rows, const int32_t* idx_local, int32_t k,
+                                int32_t n_local, int32_t offset, float* cand_score, int32_t* cand_idx, void* stream);
+size_t dsa_split_merge_workspace_bytes(int32_t n_rows, int32_t n_cand, int32_t k);
+dsa_status dsa_split_merge(const float* cand_score, const int32_t* cand_idx, int32_t n_rows, int32_t n_cand, int32_t k,
+                           int32_t lo, int32_t hi, int32_t* idx_global, int32_t* idx_local, void* workspace,
+                           size_t workspace_bytes, void* stream);
+dsa_status dsa_combine_partials(const void* o_parts, const float* lse_parts, int32_t n_parts, int32_t n_q, void* out,
+                                float* lse, void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * 78-layer schedule (ailearn "IndexShare：四层共用一次搜索结果"): Full at 0-based layers 0, 1
  * and 2 + 4g; every other layer reuses the closest preceding Full layer.
  */

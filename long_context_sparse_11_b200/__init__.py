@@ -6,6 +6,7 @@ this package is its Python binding.  Build it with ``long_context_sparse_11_b200
 from .binding import (  # noqa: F401
     CacheView, IndexHandle, GroupArgs, DsaError, IndexShareGroup, load, dense_view, paged_view,
     quant_e4m3, cache_write_e4m3, indexer_score, topk, topk_no_alloc, sparse_mla_attn, sync_status,
-    layer_is_full, layer_producer,
+    layer_is_full, layer_producer, indexer_project, mla_latent, rope_query, ROPE_THETA,
+    split_candidates, split_merge, combine_partials,
     DSA_BF16, DSA_E4M3, EXPORTS,
 )

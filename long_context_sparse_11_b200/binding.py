@@ -27,6 +27,9 @@ EXPORTS = [
     "indexshare_group_forward", "dsa_layer_is_full", "dsa_layer_producer", "dsa_status_str",
     "dsa_last_error", "dsa_abi_version", "dsa_abi_sizeof", "dsa_sync_status", "dsa_debug_bounded_wait",
     "dsa_set_wait_limit_ns", "dsa_launch_count", "dsa_topk_no_alloc", "dsa_cache_write_e4m3",
+    "dsa_indexer_project_workspace_bytes", "dsa_indexer_project", "dsa_mla_latent_workspace_bytes", "dsa_mla_latent",
+    "dsa_rope_query", "dsa_split_candidates", "dsa_split_merge_workspace_bytes", "dsa_split_merge",
+    "dsa_combine_partials",
 ]
 
 
@@ -93,6 +96,19 @@ def load(path: str = LIB_PATH):
         "dsa_launch_count": (c_int64, []),
         "dsa_topk_no_alloc": (S, [c_void_p, c_int64, c_int32, c_void_p, c_int64, c_int64, c_int32, c_void_p,
                                   c_void_p]),
+        "dsa_indexer_project_workspace_bytes": (c_size_t, [c_int32]),
+        "dsa_indexer_project": (S, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_int32,
+                                    c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+        "dsa_mla_latent_workspace_bytes": (c_size_t, [c_int32]),
+        "dsa_mla_latent": (S, [c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_float, c_void_p, c_void_p,
+                               c_size_t, c_void_p]),
+        "dsa_rope_query": (S, [c_void_p, c_void_p, c_int32, c_float, c_void_p]),
+        "dsa_split_candidates": (S, [c_void_p, c_int64, c_int32, c_void_p, c_int32, c_int32, c_int32, c_void_p,
+                                     c_void_p, c_void_p]),
+        "dsa_split_merge_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int32]),
+        "dsa_split_merge": (S, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_int32, c_int32, c_void_p, c_void_p,
+                                c_void_p, c_size_t, c_void_p]),
+        "dsa_combine_partials": (S, [c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_void_p]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -220,6 +236,87 @@ def sparse_mla_attn(q, kv: CacheView, idx, k: int, softmax_scale: float, q_rows_
     _check(lib.dsa_sparse_mla_attn(q.data_ptr(), ctypes.byref(kv), idx.data_ptr(), n_q, q_rows_per_idx_row, k,
                                    softmax_scale, out.data_ptr(), lse.data_ptr(), _ptr(workspace),
                                    0 if workspace is None else workspace.numel(), _stream()))
+    return out, lse
+
+
+ROPE_THETA = 8.0e6
+
+
+def indexer_project(cq, x, Wq, Wkw, gamma, beta, q_out=None, k_out=None, w_out=None, workspace=None):
+    """The indexer's inputs: q [T,32,128] bf16 from the query latent cq [T,q_rank], the key
+    [T,128] bf16 (LayerNorm) and head weights [T,32] fp32 from the hidden state x [T,hidden];
+    Wq [4096,q_rank], Wkw [160,hidden] (Wk rows then Ww rows) bf16, gamma / beta [128] fp32."""
+    import torch
+    T = cq.shape[0]
+    dev = cq.device
+    q_out = torch.empty(T, 32, 128, dtype=torch.bfloat16, device=dev) if q_out is None else q_out
+    k_out = torch.empty(T, 128, dtype=torch.bfloat16, device=dev) if k_out is None else k_out
+    w_out = torch.empty(T, 32, dtype=torch.float32, device=dev) if w_out is None else w_out
+    lib = load()
+    need = lib.dsa_indexer_project_workspace_bytes(T)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib.dsa_indexer_project(cq.data_ptr(), x.data_ptr(), Wq.data_ptr(), Wkw.data_ptr(), gamma.data_ptr(),
+                                   beta.data_ptr(), T, cq.shape[1], x.shape[1], q_out.data_ptr(), k_out.data_ptr(),
+                                   w_out.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream()))
+    return q_out, k_out, w_out
+
+
+def mla_latent(x, Wkv, gamma, pos, theta: float = ROPE_THETA, out=None, workspace=None):
+    """Latent KV rows [T,576] bf16 from the hidden state x [T,hidden]: RMSNorm of x W_dkv^T (512 dims)
+    and RoPE of x W_kr^T (64 dims) at positions pos [T] int32; Wkv [576,hidden] bf16, gamma [512] fp32."""
+    import torch
+    T = x.shape[0]
+    out = torch.empty(T, 576, dtype=torch.bfloat16, device=x.device) if out is None else out
+    lib = load()
+    if workspace is None:
+        workspace = torch.empty(max(lib.dsa_mla_latent_workspace_bytes(T), 16), dtype=torch.uint8, device=x.device)
+    _check(lib.dsa_mla_latent(x.data_ptr(), Wkv.data_ptr(), gamma.data_ptr(), pos.data_ptr(), T, x.shape[1], theta,
+                              out.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream()))
+    return out
+
+
+def rope_query(q, pos, theta: float = ROPE_THETA):
+    """Turn dims 512..575 of every head of q [T,64,576] bf16 in place to positions pos [T] int32."""
+    _check(load().dsa_rope_query(q.data_ptr(), pos.data_ptr(), q.shape[0], theta, _stream()))
+    return q
+
+
+def split_candidates(scores, idx_local, n_local: int, offset: int):
+    """A rank's local Top-k [rows, k] over its slice's scores [rows, ld] -> (cand_score [rows, k] fp32,
+    cand_idx [rows, k] int32): (score, offset + position) ordered by position, padding last."""
+    import torch
+    rows, k = idx_local.shape
+    cs = torch.empty(rows, k, dtype=torch.float32, device=scores.device)
+    ci = torch.empty(rows, k, dtype=torch.int32, device=scores.device)
+    _check(load().dsa_split_candidates(scores.data_ptr(), scores.stride(0), rows, idx_local.data_ptr(), k, n_local,
+                                       offset, cs.data_ptr(), ci.data_ptr(), _stream()))
+    return cs, ci
+
+
+def split_merge(cand_score, cand_idx, k: int, lo: int, hi: int, workspace=None):
+    """All ranks' candidates [rows, G*k] (rank order) -> (idx_global [rows, k], idx_local [rows, k])."""
+    import torch
+    rows, n_cand = cand_score.shape
+    ig = torch.empty(rows, k, dtype=torch.int32, device=cand_score.device)
+    il = torch.empty(rows, k, dtype=torch.int32, device=cand_score.device)
+    lib = load()
+    need = lib.dsa_split_merge_workspace_bytes(rows, n_cand, k)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=cand_score.device)
+    _check(lib.dsa_split_merge(cand_score.data_ptr(), cand_idx.data_ptr(), rows, n_cand, k, lo, hi, ig.data_ptr(),
+                               il.data_ptr(), _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream()))
+    return ig, il
+
+
+def combine_partials(o_parts, lse_parts, out=None, lse=None):
+    """Partial attention of G ranks, o_parts [G,n_q,64,512] bf16 and lse_parts [G,n_q,64] fp32 -> out, lse."""
+    import torch
+    G, n_q = lse_parts.shape[0], lse_parts.shape[1]
+    out = torch.empty(n_q, 64, 512, dtype=torch.bfloat16, device=o_parts.device) if out is None else out
+    lse = torch.empty(n_q, 64, dtype=torch.float32, device=o_parts.device) if lse is None else lse
+    _check(load().dsa_combine_partials(o_parts.data_ptr(), lse_parts.data_ptr(), G, n_q, out.data_ptr(),
+                                       _ptr(lse), _stream()))
     return out, lse
 
 

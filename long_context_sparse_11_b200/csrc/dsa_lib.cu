@@ -10,15 +10,19 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
 
 #include "../../include/dsa.h"
+#include "gemm.cuh"
 #include "indexer.cuh"
 #include "mla.cuh"
+#include "mla_pair.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
+#include "splitn.cuh"
 #include "topk.cuh"
 
 namespace dsa {
@@ -77,7 +81,18 @@ struct DeviceState {
   bool ready = false;
   int sms = 148;
   int* status = nullptr;
+  int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair attention kernel (0: not usable)
 };
+
+// Sparse MLA over a dense bf16 cache with many rows runs on CTA pairs unless DSA_MLA_PAIR=0 in the
+// environment (kept to compare the two kernels on the same inputs).
+bool pair_kernel_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("DSA_MLA_PAIR");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 DeviceState g_dev[64];
 std::mutex g_mu;
 
@@ -122,6 +137,31 @@ dsa_status device_state(DeviceState** out) {
     DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<true, true>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES),
                        "smem attr"));
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(gemm::gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            gemm::SMEM_BYTES),
+                       "smem attr"));
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(mlap::sparse_mla_pair_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, mlap::SMEM_BYTES),
+                       "smem attr"));
+    {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * static_cast<unsigned>(d.sms / 2));
+      cfg.blockDim = dim3(mlap::THREADS);
+      cfg.dynamicSmemBytes = mlap::SMEM_BYTES;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, mlap::sparse_mla_pair_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+      d.pair_clusters = n;
+    }
     DSA_TRY(cuda_check(cudaFuncSetAttribute(topk::topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             static_cast<int>(sizeof(topk::Smem))),
                        "smem attr"));
@@ -362,6 +402,42 @@ size_t mla_ws_bytes(int32_t n_q, int32_t k, int sms) {
   return static_cast<size_t>(n_q) * s * (64 * 512 * 4 + 128 * 4) + 256;
 }
 
+// Many query rows over a dense bf16 cache, one selection per row: the CTA-pair kernel.
+dsa_status launch_mla_pair(const DeviceState* ds, const void* q, const dsa_cache_view* kv, const int32_t* idx,
+                           int32_t n_q, int32_t k, float softmax_scale, void* out, float* lse, cudaStream_t st,
+                           int64_t valid0) {
+  mlap::Params p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.kv = static_cast<const uint8_t*>(kv->data);
+  p.idx = idx;
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.row_stride = kv->row_stride;
+  p.n_tokens = kv->n_tokens;
+  p.n_q = n_q;
+  p.k = k;
+  p.valid0 = valid0;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.status = ds->status;
+  p.wait_ns = static_cast<uint64_t>(g_wait_ns);
+  const int clusters = std::min(ds->pair_clusters, n_q);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * static_cast<unsigned>(clusters));
+  cfg.blockDim = dim3(mlap::THREADS);
+  cfg.dynamicSmemBytes = mlap::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  DSA_TRY(cuda_check(cudaLaunchKernelEx(&cfg, mlap::sparse_mla_pair_kernel, p), "sparse MLA pair launch"));
+  count_launch();
+  return DSA_OK;
+}
+
 dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* idx, int32_t n_q, int32_t rpi,
                       int32_t k, float softmax_scale, void* out, float* lse, void* ws, size_t ws_bytes,
                       cudaStream_t st, int64_t valid0 = -1) {
@@ -369,6 +445,8 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
   DSA_TRY(device_state(&ds));
   if (n_q == 0) return DSA_OK;
   const bool paged = kv->block_table != nullptr;
+  if (!paged && rpi == 1 && n_q >= 2 * ds->sms && ds->pair_clusters > 0 && pair_kernel_enabled())
+    return launch_mla_pair(ds, q, kv, idx, n_q, k, softmax_scale, out, lse, st, valid0);
   mla::Params p{};
   p.q = static_cast<const uint16_t*>(q);
   p.kv = static_cast<const uint8_t*>(kv->data);
@@ -424,6 +502,32 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
     DSA_TRY(cuda_check(cudaGetLastError(), "combine launch"));
   }
   return DSA_OK;
+}
+
+// C[m, n] (fp32 or bf16, row stride ldc) = A[m, k] . B[n, k]^T, A and B bf16 with rows of k.
+dsa_status launch_gemm(const void* A, const void* B, int32_t m, int32_t n, int32_t k, void* C, int64_t ldc,
+                       bool out_bf16, cudaStream_t st) {
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  if (m == 0 || n == 0) return DSA_OK;
+  CUtensorMap ma, mb;
+  DSA_TRY(make_map(&ma, A, true, static_cast<uint64_t>(k), static_cast<uint64_t>(m), static_cast<uint64_t>(k) * 2, 64,
+                   gemm::BM));
+  DSA_TRY(make_map(&mb, B, true, static_cast<uint64_t>(k), static_cast<uint64_t>(n), static_cast<uint64_t>(k) * 2, 64,
+                   gemm::BN));
+  gemm::Params p{};
+  p.c = C;
+  p.ldc = ldc;
+  p.m = m;
+  p.n = n;
+  p.k = k;
+  p.out_bf16 = out_bf16 ? 1 : 0;
+  p.status = ds->status;
+  p.wait_ns = static_cast<uint64_t>(g_wait_ns);
+  dim3 grid(static_cast<unsigned>((n + gemm::BN - 1) / gemm::BN), static_cast<unsigned>((m + gemm::BM - 1) / gemm::BM));
+  gemm::gemm_bf16_kernel<<<grid, gemm::THREADS, gemm::SMEM_BYTES, st>>>(ma, mb, p);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "projection GEMM launch");
 }
 
 // ---------------------------------------------------------------------------- group plan
@@ -600,6 +704,7 @@ dsa_status dsa_sync_status(void* stream) {
   DSA_TRY(cuda_check(cudaMemcpy(ds->status, &zero, sizeof(int), cudaMemcpyHostToDevice), "clear status"));
   if (v & DEVERR_TIMEOUT) return fail(DSA_ERR_TIMEOUT, "a bounded device wait ran out");
   if (v & DEVERR_BOUNDS) return fail(DSA_ERR_BOUNDS, "a kernel skipped an out-of-range index or page");
+  if (v & DEVERR_LAUNCH) return fail(DSA_ERR_CUDA, "a kernel was launched without the CTA cluster it needs");
   if (v & DEVERR_RANGE)
     return fail(DSA_ERR_RANGE, "a query value of an attention over an e4m3 cache exceeds the f16 range");
   return DSA_OK;
@@ -673,6 +778,125 @@ dsa_status dsa_indexer_score(const void* q, int32_t q_dtype, const float* q_scal
   }
   return launch_indexer(q, q_dtype, q_scale, w, n_q, q_pos0, keys, scores, ld_scores,
                         static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_indexer_project_workspace_bytes(int32_t n_tokens) {
+  return n_tokens <= 0 ? 0 : static_cast<size_t>(n_tokens) * 160 * 4 + 256;
+}
+
+dsa_status dsa_indexer_project(const void* cq, const void* x, const void* Wq, const void* Wkw, const float* gamma,
+                               const float* beta, int32_t n_tokens, int32_t q_rank, int32_t hidden, void* q_out,
+                               void* k_out, float* w_out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (n_tokens < 0) return fail(DSA_ERR_INVALID_ARG, "n_tokens < 0");
+  if (q_rank < 64 || q_rank % 64 || hidden < 64 || hidden % 64)
+    return fail(DSA_ERR_UNSUPPORTED, "q_rank %d / hidden %d must be positive multiples of 64", q_rank, hidden);
+  if (n_tokens == 0) return DSA_OK;
+  const void* ptrs[] = {cq, x, Wq, Wkw, gamma, beta, q_out, k_out, w_out, workspace};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return fail(DSA_ERR_INVALID_ARG, "null or misaligned pointer");
+  if (workspace_bytes < dsa_indexer_project_workspace_bytes(n_tokens))
+    return fail(DSA_ERR_WORKSPACE, "indexer projection needs %zu workspace bytes",
+                dsa_indexer_project_workspace_bytes(n_tokens));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* kw = static_cast<float*>(workspace);
+  DSA_TRY(launch_gemm(cq, Wq, n_tokens, 4096, q_rank, q_out, 4096, true, st));
+  DSA_TRY(launch_gemm(x, Wkw, n_tokens, 160, hidden, kw, 160, false, st));
+  gemm::key_norm_kernel<<<static_cast<unsigned>((n_tokens + 7) / 8), 256, 0, st>>>(
+      kw, n_tokens, gamma, beta, 1e-6f, static_cast<uint16_t*>(k_out), w_out);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "key norm launch");
+}
+
+size_t dsa_mla_latent_workspace_bytes(int32_t n_tokens) {
+  return n_tokens <= 0 ? 0 : static_cast<size_t>(n_tokens) * 576 * 4 + 256;
+}
+
+dsa_status dsa_mla_latent(const void* x, const void* Wkv, const float* gamma, const int32_t* pos, int32_t n_tokens,
+                          int32_t hidden, float theta, void* latent_out, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  if (n_tokens < 0) return fail(DSA_ERR_INVALID_ARG, "n_tokens < 0");
+  if (hidden < 64 || hidden % 64) return fail(DSA_ERR_UNSUPPORTED, "hidden %d must be a positive multiple of 64", hidden);
+  if (!(theta > 1.f)) return fail(DSA_ERR_INVALID_ARG, "theta must be > 1");
+  if (n_tokens == 0) return DSA_OK;
+  const void* ptrs[] = {x, Wkv, gamma, pos, latent_out, workspace};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return fail(DSA_ERR_INVALID_ARG, "null or misaligned pointer");
+  if (workspace_bytes < dsa_mla_latent_workspace_bytes(n_tokens))
+    return fail(DSA_ERR_WORKSPACE, "latent projection needs %zu workspace bytes", dsa_mla_latent_workspace_bytes(n_tokens));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* y = static_cast<float*>(workspace);
+  DSA_TRY(launch_gemm(x, Wkv, n_tokens, 576, hidden, y, 576, false, st));
+  gemm::latent_norm_rope_kernel<<<static_cast<unsigned>((n_tokens + 7) / 8), 256, 0, st>>>(
+      y, n_tokens, gamma, pos, 1e-6f, static_cast<double>(theta), static_cast<uint16_t*>(latent_out));
+  count_launch();
+  return cuda_check(cudaGetLastError(), "latent norm / rope launch");
+}
+
+dsa_status dsa_rope_query(void* q, const int32_t* pos, int32_t n_q, float theta, void* stream) {
+  if (n_q < 0) return fail(DSA_ERR_INVALID_ARG, "n_q < 0");
+  if (!(theta > 1.f)) return fail(DSA_ERR_INVALID_ARG, "theta must be > 1");
+  if (n_q == 0) return DSA_OK;
+  if (!q || !aligned16(q) || !pos) return fail(DSA_ERR_INVALID_ARG, "null or misaligned pointer");
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  gemm::rope_query_kernel<<<static_cast<unsigned>(n_q), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint16_t*>(q), n_q, pos, static_cast<double>(theta));
+  count_launch();
+  return cuda_check(cudaGetLastError(), "query rope launch");
+}
+
+dsa_status dsa_split_candidates(const float* scores, int64_t ld, int32_t n_rows, const int32_t* idx_local, int32_t k,
+                                int32_t n_local, int32_t offset, float* cand_score, int32_t* cand_idx, void* stream) {
+  if (k < 1 || k > DSA_MAX_K) return fail(DSA_ERR_INVALID_ARG, "k %d not in [1,2048]", k);
+  if (n_rows < 0 || n_local < 0 || offset < 0 || ld <= 0) return fail(DSA_ERR_INVALID_ARG, "bad sizes");
+  if (static_cast<int64_t>(offset) + n_local > INT32_MAX) return fail(DSA_ERR_INVALID_ARG, "positions beyond int32");
+  if (n_rows == 0) return DSA_OK;
+  if (!scores || !idx_local || !cand_score || !cand_idx) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  splitn::split_candidates_kernel<<<static_cast<unsigned>(n_rows), 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+      scores, ld, idx_local, k, offset, n_local, cand_score, cand_idx, ds->status);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "split candidates launch");
+}
+
+size_t dsa_split_merge_workspace_bytes(int32_t n_rows, int32_t n_cand, int32_t k) {
+  return dsa_topk_workspace_bytes(n_rows, n_cand, k);
+}
+
+dsa_status dsa_split_merge(const float* cand_score, const int32_t* cand_idx, int32_t n_rows, int32_t n_cand, int32_t k,
+                           int32_t lo, int32_t hi, int32_t* idx_global, int32_t* idx_local, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (k < 1 || k > DSA_MAX_K) return fail(DSA_ERR_INVALID_ARG, "k %d not in [1,2048]", k);
+  if (n_rows < 0 || n_cand < 1 || n_cand % 4 || lo < 0 || hi < lo)
+    return fail(DSA_ERR_INVALID_ARG, "bad sizes (n_cand must be a positive multiple of 4)");
+  if (n_rows == 0) return DSA_OK;
+  if (!cand_score || !aligned16(cand_score) || !cand_idx || !idx_global || !aligned16(idx_global) || !idx_local)
+    return fail(DSA_ERR_INVALID_ARG, "null or misaligned pointer");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // positions of the k best candidates of each row (every row holds n_cand: row length
+  // causal_len0 + r capped at n_cand), written into idx_global, then mapped in place
+  DSA_TRY(launch_topk(cand_score, n_cand, n_rows, nullptr, n_cand, n_cand, k, idx_global, workspace, workspace_bytes,
+                      st));
+  const int64_t total = static_cast<int64_t>(n_rows) * k;
+  splitn::split_map_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(cand_idx, n_cand, k, n_rows,
+                                                                                    idx_global, idx_local, lo, hi);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "split map launch");
+}
+
+dsa_status dsa_combine_partials(const void* o_parts, const float* lse_parts, int32_t n_parts, int32_t n_q, void* out,
+                                float* lse, void* stream) {
+  if (n_parts < 1 || n_q < 0) return fail(DSA_ERR_INVALID_ARG, "bad sizes");
+  if (n_q == 0) return DSA_OK;
+  if (!o_parts || !aligned16(o_parts) || !lse_parts || !out || !aligned16(out))
+    return fail(DSA_ERR_INVALID_ARG, "null or misaligned pointer");
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  splitn::combine_parts_kernel<<<dim3(static_cast<unsigned>(n_q), 64), 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(o_parts), lse_parts, n_parts, n_q, static_cast<uint16_t*>(out), lse);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "combine launch");
 }
 
 size_t dsa_topk_workspace_bytes(int32_t n_rows, int64_t max_len, int32_t k) {

@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
         // head sum of one query from registers: ReLU, per-head weight, packed FMA on head pairs
         auto score = [&](const uint32_t (&x)[32], int qq) {
           const float4* wv = reinterpret_cast<const float4*>(w_s + (g * C::NQ + qq) * 32);
-          float a0 = 0.f, a1 = 0.f;
+          float2 a2 = make_float2(0.f, 0.f);
 #pragma unroll
           for (int h4 = 0; h4 < 8; ++h4) {
             const float4 ww = wv[h4];
@@ -295,10 +295,11 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
               const float v = __uint_as_float(x[4 * h4 + u]);
               r[u] = relu_on_fma<C::RELU_FMA_PAIRS>(2 * h4 + u / 2) ? v + fabsf(v) : fmaxf(v, 0.f);
             }
-            ffma2(a0, a1, ww.x, ww.y, r[0], r[1]);
-            ffma2(a0, a1, ww.z, ww.w, r[2], r[3]);
+            // packed fp32 FMA on head pairs (the compiler's own pairing of the operands)
+            a2 = __ffma2_rn(make_float2(ww.x, ww.y), make_float2(r[0], r[1]), a2);
+            a2 = __ffma2_rn(make_float2(ww.z, ww.w), make_float2(r[2], r[3]), a2);
           }
-          float acc = a0 + a1;
+          float acc = a2.x + a2.y;
           if (FP8) acc *= sk;
           if (PAGED) {
             if (s_abs < len) p.scores[static_cast<int64_t>(b) * p.ld + s_abs] = acc;

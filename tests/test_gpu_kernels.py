@@ -302,6 +302,34 @@ def test_sparse_mla_dense_bf16(L, k):
         assert np.max(np.abs(l[r] - ref_l[r])) <= 2e-3
 
 
+@pytest.mark.parametrize("L,k", [(700, 200), (3000, 2048)])
+def test_sparse_mla_dense_bf16_many_rows(L, k):
+    """At least 2 rows per SM: the rows run on CTA pairs that split each latent row by its dims
+    (the prefill kernel); checked like the test above, with padding inside rows as well."""
+    n_q = 400
+    Qb = bf16_bits_np(normal_np(51, 0, n_q * 64 * 576)).reshape(n_q, 64, 576)
+    KVb = bf16_bits_np(normal_np(52, 0, L * 576)).reshape(L, 576)
+    sc = normal_np(53, 0, n_q * L).reshape(n_q, L)
+    idx = np.stack([O.topk_row(sc[r], min(L, L - n_q + r + 1), k) for r in range(n_q)]).astype(np.int32)
+    idx[7, :] = -1                                              # an empty row
+    idx[11, 3::5] = -1                                          # padding scattered inside a row
+    idx[12, 130:] = -1                                          # a row that ends inside its second tile
+    out, lse = dsa.sparse_mla_attn(bf16_dev(Qb), dsa.dense_view(bf16_dev(KVb)), i32_dev(idx), k, SCALE)
+    dsa.sync_status()
+    o = O.bf16_to_f64(bf16_host(out))
+    l = lse.cpu().numpy()
+    Q, KV = O.bf16_to_f64(Qb), O.bf16_to_f64(KVb)
+    rows = sorted(set(list(range(0, n_q, 13)) + [11, 12, n_q - 1]))
+    ref_o, ref_l = _mla_ref(Q, KV, idx, rows)
+    for r in rows + [7]:
+        if r == 7:
+            assert np.all(o[r] == 0) and np.all(np.isneginf(l[r]))
+            continue
+        ma, rl = attn_errors(o[r], ref_o[r])
+        assert ma <= 2e-2 and rl <= 5e-3, (r, ma, rl)
+        assert np.max(np.abs(l[r] - ref_l[r])) <= 2e-3
+
+
 def test_sparse_mla_k_covers_history_is_dense():
     L = 200
     Qb = bf16_bits_np(normal_np(41, 0, L * 64 * 576)).reshape(L, 64, 576)
