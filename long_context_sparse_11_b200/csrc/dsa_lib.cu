@@ -10,7 +10,6 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -19,7 +18,6 @@
 #include "gemm.cuh"
 #include "indexer.cuh"
 #include "mla.cuh"
-#include "mla_pair.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 #include "splitn.cuh"
@@ -81,18 +79,8 @@ struct DeviceState {
   bool ready = false;
   int sms = 148;
   int* status = nullptr;
-  int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair attention kernel (0: not usable)
 };
 
-// Sparse MLA over a dense bf16 cache with many rows runs on CTA pairs unless DSA_MLA_PAIR=0 in the
-// environment (kept to compare the two kernels on the same inputs).
-bool pair_kernel_enabled() {
-  static const bool on = [] {
-    const char* e = std::getenv("DSA_MLA_PAIR");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
 DeviceState g_dev[64];
 std::mutex g_mu;
 
@@ -140,28 +128,6 @@ dsa_status device_state(DeviceState** out) {
     DSA_TRY(cuda_check(cudaFuncSetAttribute(gemm::gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             gemm::SMEM_BYTES),
                        "smem attr"));
-    DSA_TRY(cuda_check(cudaFuncSetAttribute(mlap::sparse_mla_pair_kernel,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize, mlap::SMEM_BYTES),
-                       "smem attr"));
-    {
-      cudaLaunchConfig_t cfg = {};
-      cudaLaunchAttribute at[1];
-      at[0].id = cudaLaunchAttributeClusterDimension;
-      at[0].val.clusterDim.x = 2;
-      at[0].val.clusterDim.y = 1;
-      at[0].val.clusterDim.z = 1;
-      cfg.gridDim = dim3(2 * static_cast<unsigned>(d.sms / 2));
-      cfg.blockDim = dim3(mlap::THREADS);
-      cfg.dynamicSmemBytes = mlap::SMEM_BYTES;
-      cfg.attrs = at;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, mlap::sparse_mla_pair_kernel, &cfg) != cudaSuccess) {
-        cudaGetLastError();
-        n = 0;
-      }
-      d.pair_clusters = n;
-    }
     DSA_TRY(cuda_check(cudaFuncSetAttribute(topk::topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             static_cast<int>(sizeof(topk::Smem))),
                        "smem attr"));
@@ -402,42 +368,6 @@ size_t mla_ws_bytes(int32_t n_q, int32_t k, int sms) {
   return static_cast<size_t>(n_q) * s * (64 * 512 * 4 + 128 * 4) + 256;
 }
 
-// Many query rows over a dense bf16 cache, one selection per row: the CTA-pair kernel.
-dsa_status launch_mla_pair(const DeviceState* ds, const void* q, const dsa_cache_view* kv, const int32_t* idx,
-                           int32_t n_q, int32_t k, float softmax_scale, void* out, float* lse, cudaStream_t st,
-                           int64_t valid0) {
-  mlap::Params p{};
-  p.q = static_cast<const uint16_t*>(q);
-  p.kv = static_cast<const uint8_t*>(kv->data);
-  p.idx = idx;
-  p.out = static_cast<uint16_t*>(out);
-  p.lse = lse;
-  p.row_stride = kv->row_stride;
-  p.n_tokens = kv->n_tokens;
-  p.n_q = n_q;
-  p.k = k;
-  p.valid0 = valid0;
-  p.scale_log2 = softmax_scale * 1.4426950408889634f;
-  p.status = ds->status;
-  p.wait_ns = static_cast<uint64_t>(g_wait_ns);
-  const int clusters = std::min(ds->pair_clusters, n_q);
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = 2;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(2 * static_cast<unsigned>(clusters));
-  cfg.blockDim = dim3(mlap::THREADS);
-  cfg.dynamicSmemBytes = mlap::SMEM_BYTES;
-  cfg.stream = st;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  DSA_TRY(cuda_check(cudaLaunchKernelEx(&cfg, mlap::sparse_mla_pair_kernel, p), "sparse MLA pair launch"));
-  count_launch();
-  return DSA_OK;
-}
-
 dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* idx, int32_t n_q, int32_t rpi,
                       int32_t k, float softmax_scale, void* out, float* lse, void* ws, size_t ws_bytes,
                       cudaStream_t st, int64_t valid0 = -1) {
@@ -445,8 +375,6 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
   DSA_TRY(device_state(&ds));
   if (n_q == 0) return DSA_OK;
   const bool paged = kv->block_table != nullptr;
-  if (!paged && rpi == 1 && n_q >= 2 * ds->sms && ds->pair_clusters > 0 && pair_kernel_enabled())
-    return launch_mla_pair(ds, q, kv, idx, n_q, k, softmax_scale, out, lse, st, valid0);
   mla::Params p{};
   p.q = static_cast<const uint16_t*>(q);
   p.kv = static_cast<const uint8_t*>(kv->data);
@@ -704,7 +632,6 @@ dsa_status dsa_sync_status(void* stream) {
   DSA_TRY(cuda_check(cudaMemcpy(ds->status, &zero, sizeof(int), cudaMemcpyHostToDevice), "clear status"));
   if (v & DEVERR_TIMEOUT) return fail(DSA_ERR_TIMEOUT, "a bounded device wait ran out");
   if (v & DEVERR_BOUNDS) return fail(DSA_ERR_BOUNDS, "a kernel skipped an out-of-range index or page");
-  if (v & DEVERR_LAUNCH) return fail(DSA_ERR_CUDA, "a kernel was launched without the CTA cluster it needs");
   if (v & DEVERR_RANGE)
     return fail(DSA_ERR_RANGE, "a query value of an attention over an e4m3 cache exceeds the f16 range");
   return DSA_OK;

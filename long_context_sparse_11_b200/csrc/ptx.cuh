@@ -8,7 +8,7 @@
 namespace dsa {
 
 // Device-side status word bits (read back by dsa_sync_status).
-enum : int { DEVERR_TIMEOUT = 1, DEVERR_BOUNDS = 2, DEVERR_RANGE = 4, DEVERR_LAUNCH = 8 };
+enum : int { DEVERR_TIMEOUT = 1, DEVERR_BOUNDS = 2, DEVERR_RANGE = 4 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -62,97 +62,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
   }
   return true;
-}
-
-// The same wait, with acquire semantics at cluster scope: for barriers that threads of another
-// CTA of the cluster arrive on (remotely, with release at cluster scope) after writing this
-// CTA's shared memory.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
-                                                  uint64_t limit_ns) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait_cluster(bar, parity)) {
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      *abort = 1;
-      atomicOr(status, DEVERR_TIMEOUT);
-      return false;
-    }
-  }
-  return true;
-}
-
-// ---------------------------------------------------------------------------- thread-block clusters
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_size() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_id_x() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_count_x() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
-  return r;
-}
-// Address, in the cluster's shared window, of the same shared-memory location in CTA `rank`.
-__device__ __forceinline__ uint32_t map_to_cta(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void st_cluster_v4(uint32_t caddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
-__device__ __forceinline__ void st_cluster_f32(uint32_t caddr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(caddr), "f"(v) : "memory");
-}
-__device__ __forceinline__ void st_cluster_u32(uint32_t caddr, uint32_t v) {
-  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
-}
-// Asynchronous store into another CTA's shared memory whose completion is counted (in bytes)
-// on an mbarrier of that CTA (complete_tx): the receiver arms the barrier with the bytes it
-// expects and waits on it like on a TMA load, with no cluster-scope fence on either side.
-__device__ __forceinline__ void st_async_v4(uint32_t caddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                                            uint32_t cbar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                   caddr),
-               "r"(a), "r"(b), "r"(c), "r"(d), "r"(cbar)
-               : "memory");
-}
-__device__ __forceinline__ void st_async_b32(uint32_t caddr, uint32_t v, uint32_t cbar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(caddr), "r"(v),
-               "r"(cbar)
-               : "memory");
-}
-// Arrive on an mbarrier of another CTA of the cluster; this thread's earlier writes (and those
-// ordered before them) are released to that CTA's acquiring waiters.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
-}
-// All threads of every CTA of the cluster: arrive and wait (release / acquire at cluster scope).
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------- barriers / fences
@@ -237,14 +146,6 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-// Arrive once on the mbarrier at this shared offset in every CTA of cta_mask when all previously
-// issued tcgen05 ops of this thread complete.
-__device__ __forceinline__ void mma_commit_multicast(uint32_t bar, uint16_t cta_mask) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-               ::"r"(bar), "h"(cta_mask)
-               : "memory");
-}
-
 // Instruction descriptor (kind::f16 / kind::f8f6f4), f32 accumulator.
 // fmt: kind::f16 -> 0 = f16, 1 = bf16; kind::f8f6f4 -> 0 = e4m3.  mn_major: 0 = K-major.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t a_fmt, uint32_t b_fmt, uint32_t a_mn, uint32_t b_mn,
@@ -263,18 +164,6 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo_byte
   d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;  // descriptor version for sm_100
   d |= (uint64_t)2 << 61;  // SWIZZLE_128B
-  return d;
-}
-
-// Shared-memory matrix descriptor without swizzle (K-major "interleaved" layout): 8-row x 16-byte
-// core matrices stored as 128 contiguous bytes; lbo = byte stride between core matrices along K,
-// sbo = byte stride between them along M/N.
-__device__ __forceinline__ uint64_t make_sdesc_noswz(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;  // descriptor version for sm_100; layout type 0 = no swizzle
   return d;
 }
 
@@ -315,21 +204,6 @@ __host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c) {
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])  \
       : "r"(taddr)                                                                                            \
       : "memory")
-
-#define DSA_TMEM_LD_X8_NOWAIT(taddr, r)                                                                       \
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"                          \
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]) \
-               : "r"(taddr)                                                                                   \
-               : "memory")
-// Waits for all of the thread's outstanding TMEM loads; names both destinations so that no use of
-// either is scheduled before it.
-#define DSA_TMEM_WAIT_LD_X8X2(a, b)                                                                           \
-  asm volatile("tcgen05.wait::ld.sync.aligned;"                                                               \
-               : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]),         \
-                 "+r"(a[7]), "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]),          \
-                 "+r"(b[6]), "+r"(b[7])                                                                       \
-               :                                                                                              \
-               : "memory")
 
 #define DSA_TMEM_ST_X16(taddr, r)                                                                             \
   asm volatile(                                                                                               \

@@ -304,8 +304,9 @@ def test_sparse_mla_dense_bf16(L, k):
 
 @pytest.mark.parametrize("L,k", [(700, 200), (3000, 2048)])
 def test_sparse_mla_dense_bf16_many_rows(L, k):
-    """At least 2 rows per SM: the rows run on CTA pairs that split each latent row by its dims
-    (the prefill kernel); checked like the test above, with padding inside rows as well."""
+    """At least 2 rows per SM: every persistent CTA takes whole rows in turn and writes them
+    directly (no key splits, no combine pass: the prefill schedule); checked like the test
+    above, with padding inside rows as well."""
     n_q = 400
     Qb = bf16_bits_np(normal_np(51, 0, n_q * 64 * 576)).reshape(n_q, 64, 576)
     KVb = bf16_bits_np(normal_np(52, 0, L * 576)).reshape(L, 576)
