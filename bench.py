@@ -123,7 +123,7 @@ def workload_config(name, seq_len=None):
         cfg = {"workload": name, "batch": spec.batch, "context": f"U[{spec.ctx_lo},{spec.ctx_hi}]",
                "rows_per_seq": spec.rows_per_seq, "k": spec.k, "layers": spec.n_layers,
                "cache": "paged e4m3 (64-token pages), device-resident across steps; the step writes its "
-                        "current token's rows first (one launch per pool)", "indexer": "e4m3",
+                        "current token's rows into every pool first (one launch)", "indexer": "e4m3",
                "topk": "one per query row" if spec.topk_per_row else "row 0's, reused by the draft rows"}
         if spec.n_layers > 4:
             cfg["schedule"] = "Full at layers 0, 1, 2+4g; 21 groups per step"
@@ -196,6 +196,7 @@ class Workload:
                 # a decode step's new inputs: the indexer query and weights, the MLA query rows
                 self.step_inputs += [ind["q_idx"], ind["w"]] + list(inp["Q"][f:e])
             self.step_inputs += [x for x, _, _ in self.writes]     # and the current token's rows
+            self.write_all = dsa.CacheWriteBatch(self.writes, self.pos, self.bt)   # one launch per step
             self.counts = algorithmic_counts(spec, inp["ctx"])
         else:
             inp = make_prefill(spec, device=dev)
@@ -214,9 +215,8 @@ class Workload:
         return [t for g in self.groups for t in g.out + g.lse]
 
     def forward(self):
-        import long_context_sparse_11_b200 as dsa
-        for x, pool, scale in self.writes:
-            dsa.cache_write_e4m3(x, self.pos, self.bt, pool, scale)
+        if self.writes:
+            self.write_all()
         for g in self.groups:
             g.forward()
 
@@ -256,6 +256,45 @@ def indexer_alone(wl, spec, dev, stream):
     ms = e0.elapsed_time(e1)
     del scores
     return ms, (L + R - 1) // R
+
+
+def input_projections(L, dev, stream, reps=3):
+    """The steps that produce the path's inputs for L tokens, timed alone: the indexer projections
+    (q from a 2,048-rank query latent, LayerNorm key and head weights from the 6,144-wide hidden
+    state) and the latent KV rows (rank-512 compression + RMSNorm, 64 RoPE dims), on seeded random
+    bf16 weights of those shapes.  Returns their times and tensor-pipe throughput."""
+    import torch
+    import long_context_sparse_11_b200 as dsa
+    g = torch.Generator(device=dev).manual_seed(11)
+
+    def rnd(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g, device=dev) * std).to(torch.bfloat16)
+    cq, x = rnd(L, 2048), rnd(L, 6144)
+    Wq, Wkw, Wkv = rnd(4096, 2048, std=2048 ** -0.5), rnd(160, 6144, std=6144 ** -0.5), rnd(576, 6144, std=6144 ** -0.5)
+    gamma, beta, rms = (torch.ones(128, device=dev), torch.zeros(128, device=dev), torch.ones(512, device=dev))
+    pos = torch.arange(L, dtype=torch.int32, device=dev)
+    q_out, k_out, w_out = dsa.indexer_project(cq, x, Wq, Wkw, gamma, beta)
+    lat = dsa.mla_latent(x, Wkv, rms, pos)
+    res = {}
+    for name, fn, flops in (
+            ("indexer_projections", lambda: dsa.indexer_project(cq, x, Wq, Wkw, gamma, beta, q_out, k_out, w_out),
+             2.0 * L * (2048 * 4096 + 6144 * 160)),
+            ("latent_rows", lambda: dsa.mla_latent(x, Wkv, rms, pos, out=lat), 2.0 * L * 6144 * 576)):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        res[name] = {"ms": round(ms, 4), "tflops": round(flops / (ms / 1e3) / 1e12, 1)}
+    dsa.sync_status()
+    del cq, x, Wq, Wkw, Wkv, q_out, k_out, w_out, lat
+    gc.collect()
+    torch.cuda.empty_cache()
+    return res
 
 
 def independent_full_layers(wl, spec, stream, flush, reps=3):
@@ -608,6 +647,11 @@ def measure(name, args, ws, rank, local, headline):
                                    "peak": round(ia_peak, 1), "frac": round(ia_tf / ia_peak, 4),
                                    "peak_source": f"{peak_kind} bf16 dense (burst)" +
                                    (" x 2 (fp8 / bf16 nominal)" if wl.spec.indexer_fp8 else "")}
+        proj = input_projections(wl.spec.L, dev, stream)
+        for v in proj.values():
+            v.update({"peak": bf16_peak, "frac": round(v["tflops"] / bf16_peak, 4),
+                      "peak_source": f"{peak_kind} bf16 dense (burst)"})
+        phases["input_projections"] = proj
         # the IndexShare group against the same sequence run as 4 independent Full layers, both timed
         full_ms = independent_full_layers(wl, wl.spec, stream, flush)
         phases["indexshare_vs_independent_full_layers"] = {

@@ -135,6 +135,18 @@ dsa_status dsa_cache_write_e4m3(const void* x_bf16, int32_t n_rows, int32_t dim,
                                 const int32_t* pos, const int32_t* block_table, int32_t batch, int32_t max_pages,
                                 int32_t n_pages, uint8_t* pool, float* pool_scale, void* stream);
 
+/* The same write into several pools in one launch (a decode step appends its current token to
+ * every layer's latent pool and every Full layer's key pool).  x_bf16, dims, pools and
+ * pool_scales are HOST arrays of n_pools entries (device pointers inside; dims 128 or 576); all
+ * pools share seq, pos, block_table, batch, max_pages and n_pages.  n_pools <= 128.  Errors as
+ * above, per pool.
+ */
+#define DSA_CACHE_WRITE_MAX_POOLS 128
+dsa_status dsa_cache_write_e4m3_pools(int32_t n_pools, const void* const* x_bf16, const int32_t* dims,
+                                      uint8_t* const* pools, float* const* pool_scales, int32_t n_rows,
+                                      const int32_t* seq, const int32_t* pos, const int32_t* block_table, int32_t batch,
+                                      int32_t max_pages, int32_t n_pages, void* stream);
+
 /* ---------------------------------------------------------------------------------------
  * Steps a2+a3: lightweight-indexer scores (forum.sourcefind.cn "IndexShare：省掉3/4的索引计算";
  * 32 heads, ailearn architecture card), with the ReLU, per-head weight and causal mask

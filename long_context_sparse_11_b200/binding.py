@@ -29,7 +29,7 @@ EXPORTS = [
     "dsa_set_wait_limit_ns", "dsa_launch_count", "dsa_topk_no_alloc", "dsa_cache_write_e4m3",
     "dsa_indexer_project_workspace_bytes", "dsa_indexer_project", "dsa_mla_latent_workspace_bytes", "dsa_mla_latent",
     "dsa_rope_query", "dsa_split_candidates", "dsa_split_merge_workspace_bytes", "dsa_split_merge",
-    "dsa_combine_partials",
+    "dsa_combine_partials", "dsa_cache_write_e4m3_pools",
 ]
 
 
@@ -109,6 +109,8 @@ def load(path: str = LIB_PATH):
         "dsa_split_merge": (S, [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_int32, c_int32, c_void_p, c_void_p,
                                 c_void_p, c_size_t, c_void_p]),
         "dsa_combine_partials": (S, [c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p, c_void_p]),
+        "dsa_cache_write_e4m3_pools": (S, [c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_int32, c_void_p,
+                                           c_void_p, c_void_p, c_int32, c_int32, c_int32, c_void_p]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -186,6 +188,30 @@ def cache_write_e4m3(x, pos, block_table, pool, pool_scale, seq=None):
                                        block_table.shape[0], block_table.shape[1], pool.shape[0], pool.data_ptr(),
                                        pool_scale.data_ptr(), _stream()))
     return pool, pool_scale
+
+
+class CacheWriteBatch:
+    """The current token's rows of one decode step into several paged e4m3 pools with one launch:
+    writes[i] = (x [n,dim] bf16, pool [n_pages,64,dim] uint8, scale [n_pages,64] fp32), all over the
+    same block_table [B,max_pages] int32 and positions pos [n] int32 (row r -> sequence seq[r], or r).
+    The host-side pointer arrays are built once, here."""
+
+    def __init__(self, writes, pos, block_table, seq=None):
+        n = len(writes)
+        self.n_rows = writes[0][0].shape[0]
+        self.xs = (c_void_p * n)(*[x.data_ptr() for x, _, _ in writes])
+        self.dims = (c_int32 * n)(*[x.shape[1] for x, _, _ in writes])
+        self.pools = (c_void_p * n)(*[p.data_ptr() for _, p, _ in writes])
+        self.scales = (c_void_p * n)(*[s.data_ptr() for _, _, s in writes])
+        self.n_pages = writes[0][1].shape[0]
+        self.pos, self.block_table, self.seq = pos, block_table, seq
+        self._keep = writes
+
+    def __call__(self):
+        _check(load().dsa_cache_write_e4m3_pools(len(self._keep), self.xs, self.dims, self.pools, self.scales,
+                                                 self.n_rows, _ptr(self.seq), self.pos.data_ptr(),
+                                                 self.block_table.data_ptr(), self.block_table.shape[0],
+                                                 self.block_table.shape[1], self.n_pages, _stream()))
 
 
 def indexer_score(q, w, keys: CacheView, scores, q_scale=None, q_pos0: int = 0):

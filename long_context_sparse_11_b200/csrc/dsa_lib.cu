@@ -79,6 +79,7 @@ struct DeviceState {
   bool ready = false;
   int sms = 148;
   int* status = nullptr;
+  int paged_indexer_ctas_per_sm = 1;  // resident CTAs of the paged indexer kernel per SM
 };
 
 DeviceState g_dev[64];
@@ -113,6 +114,12 @@ dsa_status device_state(DeviceState** out) {
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             idx::Cfg<true, true>::SMEM_BYTES),
                        "smem attr"));
+    DSA_TRY(cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.paged_indexer_ctas_per_sm,
+                                                                     idx::indexer_kernel<true, true>,
+                                                                     idx::Cfg<true, true>::THREADS,
+                                                                     idx::Cfg<true, true>::SMEM_BYTES),
+                       "occupancy"));
+    d.paged_indexer_ctas_per_sm = std::max(1, d.paged_indexer_ctas_per_sm);
     DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<false, false>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES),
                        "smem attr"));
@@ -203,7 +210,7 @@ dsa_status check_view(const dsa_cache_view* v, int32_t dim, const char* name) {
 
 dsa_status launch_indexer(const void* q, int32_t q_dtype, const float* q_scale, const float* w, int32_t n_q,
                           int32_t q_pos0, const dsa_cache_view* keys, float* scores, int64_t ld,
-                          cudaStream_t st) {
+                          cudaStream_t st, uint32_t* hist = nullptr) {
   DeviceState* ds = nullptr;
   DSA_TRY(device_state(&ds));
   const bool fp8 = q_dtype == DSA_E4M3;
@@ -224,6 +231,7 @@ dsa_status launch_indexer(const void* q, int32_t q_dtype, const float* q_scale, 
   p.status = ds->status;
   p.wait_ns = static_cast<uint64_t>(g_wait_ns);
   p.unit_tiles = idx::UNIT_TILES;
+  p.hist = keys->block_table ? hist : nullptr;
   CUtensorMap mq, mk;
   const uint64_t qrows = static_cast<uint64_t>(n_q) * 32;
   if (paged) {
@@ -231,9 +239,16 @@ dsa_status launch_indexer(const void* q, int32_t q_dtype, const float* q_scale, 
     DSA_TRY(make_map(&mk, keys->data, false, 128, static_cast<uint64_t>(keys->n_tokens), 128, 128, 64));
     const int64_t max_len = static_cast<int64_t>(keys->max_pages) * DSA_PAGE;
     const int64_t tiles = (max_len + idx::BLOCK_KEYS - 1) / idx::BLOCK_KEYS;
-    // few long sequences: shorter units, so that the grid still covers the SMs several times over
+    // few long sequences: cut each into units so that the CTAs fill the GPU's resident slots a
+    // whole number of times (a partial last wave left a 1M-token sequence at 0.47 of HBM); many
+    // sequences keep 32-tile units, fine-grained enough to balance their different lengths
     int32_t unit = idx::UNIT_TILES;
-    while (unit > 4 && static_cast<int64_t>(n_q) * ((tiles + unit - 1) / unit) < 4LL * ds->sms) unit /= 2;
+    const int64_t slots = static_cast<int64_t>(ds->paged_indexer_ctas_per_sm) * ds->sms;
+    if (static_cast<int64_t>(n_q) * ((tiles + unit - 1) / unit) < 4 * slots) {
+      const int64_t waves = std::max<int64_t>(1, (static_cast<int64_t>(n_q) * tiles + 64 * slots - 1) / (64 * slots));
+      unit = static_cast<int32_t>(std::max<int64_t>(4, (static_cast<int64_t>(n_q) * tiles + waves * slots - 1) /
+                                                       (waves * slots)));
+    }
     p.unit_tiles = unit;
     dim3 grid(static_cast<unsigned>((tiles + unit - 1) / unit), static_cast<unsigned>(n_q));
     using C = idx::Cfg<true, true>;
@@ -289,9 +304,12 @@ TopkPlan plan_topk(int32_t n_rows, int64_t max_len, int32_t k, int sms) {
   return pl;
 }
 
+// hist_ready: the caller zeroed the workspace head (histograms + counters) and filled the
+// first-digit histograms itself (the paged indexer does, in its epilogue), so the segmented plan
+// skips its histogram pass.
 dsa_status launch_topk(const float* scores, int64_t ld, int32_t n_rows, const int32_t* row_len,
                        int64_t causal_len0, int64_t max_len, int32_t k, int32_t* idx_out, void* ws,
-                       size_t ws_bytes, cudaStream_t st) {
+                       size_t ws_bytes, cudaStream_t st, bool hist_ready = false) {
   DeviceState* ds = nullptr;
   DSA_TRY(device_state(&ds));
   const int64_t cap = std::min(ld, max_len);
@@ -312,15 +330,18 @@ dsa_status launch_topk(const float* scores, int64_t ld, int32_t n_rows, const in
   sw.cand_key = reinterpret_cast<uint32_t*>(b + head);
   sw.cand_idx = reinterpret_cast<int32_t*>(b + head + static_cast<size_t>(n_rows) * pl.gcap * 4);
   sw.gcap = pl.gcap;
-  DSA_TRY(cuda_check(cudaMemsetAsync(ws, 0, head, st), "topk workspace clear"));
   dim3 grid(pl.segs, n_rows);
-  topk::topk_seg_hist_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k,
-                                                                 pl.seg_len, sw);
+  if (!hist_ready) {
+    DSA_TRY(cuda_check(cudaMemsetAsync(ws, 0, head, st), "topk workspace clear"));
+    topk::topk_seg_hist_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k,
+                                                                   pl.seg_len, sw);
+    count_launch();
+  }
   topk::topk_seg_filter_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k,
                                                                    pl.seg_len, sw, idx_out);
   topk::topk_seg_resolve_kernel<<<n_rows, topk::THREADS, sizeof(topk::Smem), st>>>(scores, ld, row_len,
                                                                                   causal_len0, cap, k, sw, idx_out);
-  count_launch(3);
+  count_launch(2);
   return cuda_check(cudaGetLastError(), "topk launch");
 }
 
@@ -683,6 +704,36 @@ dsa_status dsa_cache_write_e4m3(const void* x_bf16, int32_t n_rows, int32_t dim,
   return cuda_check(cudaGetLastError(), "cache write launch");
 }
 
+dsa_status dsa_cache_write_e4m3_pools(int32_t n_pools, const void* const* x_bf16, const int32_t* dims,
+                                      uint8_t* const* pools, float* const* pool_scales, int32_t n_rows,
+                                      const int32_t* seq, const int32_t* pos, const int32_t* block_table, int32_t batch,
+                                      int32_t max_pages, int32_t n_pages, void* stream) {
+  if (n_pools < 0 || n_pools > CACHE_WRITE_MAX_POOLS)
+    return fail(DSA_ERR_INVALID_ARG, "n_pools %d not in [0, %d]", n_pools, CACHE_WRITE_MAX_POOLS);
+  if (n_rows < 0 || batch < 0 || max_pages < 0 || n_pages < 0) return fail(DSA_ERR_INVALID_ARG, "negative size");
+  if (n_rows == 0 || n_pools == 0) return DSA_OK;
+  if (!x_bf16 || !dims || !pools || !pool_scales || !pos || !block_table)
+    return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (batch == 0 || max_pages == 0 || n_pages == 0) return fail(DSA_ERR_INVALID_ARG, "empty cache");
+  CacheWritePools pp{};
+  for (int32_t i = 0; i < n_pools; ++i) {
+    if (dims[i] != 128 && dims[i] != 576) return fail(DSA_ERR_UNSUPPORTED, "pool %d: dim %d (128 or 576)", i, dims[i]);
+    if (!x_bf16[i] || !aligned16(x_bf16[i]) || !pools[i] || !aligned16(pools[i]) || !pool_scales[i])
+      return fail(DSA_ERR_INVALID_ARG, "pool %d: null or misaligned pointer", i);
+    pp.x[i] = static_cast<const uint16_t*>(x_bf16[i]);
+    pp.pool[i] = pools[i];
+    pp.scale[i] = pool_scales[i];
+    pp.dim[i] = dims[i];
+  }
+  DeviceState* ds = nullptr;
+  DSA_TRY(device_state(&ds));
+  const dim3 grid(static_cast<unsigned>((static_cast<int64_t>(n_rows) + 7) / 8), static_cast<unsigned>(n_pools));
+  cache_write_e4m3_pools_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      pp, n_rows, seq, pos, block_table, batch, max_pages, n_pages, ds->status);
+  count_launch();
+  return cuda_check(cudaGetLastError(), "cache write launch");
+}
+
 dsa_status dsa_indexer_score(const void* q, int32_t q_dtype, const float* q_scale, const float* w, int32_t n_q,
                              int32_t q_pos0, const dsa_cache_view* keys, float* scores, int64_t ld_scores,
                              void* stream) {
@@ -939,11 +990,18 @@ dsa_status indexshare_group_forward(const dsa_group_args* a, dsa_index_handle* h
       const int32_t c0 = ch.row0, cn = ch.rows;
       const uint8_t* qc = static_cast<const uint8_t*>(qi) + static_cast<size_t>(c0) * qrow_bytes;
       const float* qsc = qs ? qs + static_cast<size_t>(c0) * 32 : nullptr;
+      // paged rows with a segmented Top-k: the indexer's epilogue builds the first-digit
+      // histograms, so the Top-k skips that pass over the scores
+      const TopkPlan tp = plan_topk(cn, std::min<int64_t>(ch.ld, ch.max_len), a->k, ds->sms);
+      const bool fused_hist = paged && tp.segmented;
+      if (fused_hist)
+        DSA_TRY(cuda_check(cudaMemsetAsync(ws + g.off_topk, 0, static_cast<size_t>(cn) * (topk::BINS * 4 + 16), st),
+                           "topk workspace clear"));
       DSA_TRY(launch_indexer(qc, qdt, qsc, a->w + static_cast<size_t>(c0) * 32, cn, a->q_pos0 + c0, &keys, scores,
-                             ch.ld, st));
+                             ch.ld, st, fused_hist ? reinterpret_cast<uint32_t*>(ws + g.off_topk) : nullptr));
       DSA_TRY(launch_topk(scores, ch.ld, cn, paged ? keys.seq_lens : nullptr,
                           static_cast<int64_t>(a->q_pos0) + c0 + 1, ch.max_len, a->k,
-                          h->idx + static_cast<size_t>(c0) * a->k, ws + g.off_topk, g.topk_ws, st));
+                          h->idx + static_cast<size_t>(c0) * a->k, ws + g.off_topk, g.topk_ws, st, fused_hist));
     }
     h->generation += 1;
     h->filled = 1;

@@ -48,7 +48,8 @@ struct Cfg {
   static constexpr int TMEM_COLS = PAGED ? 128 : 512;
   static constexpr int KH = FP8 ? 1 : 2;          // 128-byte K halves per row
   static constexpr int KSTEPS = FP8 ? 4 : 8;
-  static constexpr int STAGES = FP8 ? 4 : 2;
+  // decode keeps 3 stages so that its 16 KB score histogram still leaves room for 3 CTAs per SM
+  static constexpr int STAGES = PAGED ? 3 : (FP8 ? 4 : 2);
   static constexpr int EPI_WARPS = PAGED ? 4 : 16;
   static constexpr int RELU_FMA_PAIRS = FP8 ? DSA_IDX_RELU_FMA_PAIRS_E4M3 : DSA_IDX_RELU_FMA_PAIRS_BF16;
   static constexpr int THREADS = 64 + EPI_WARPS * 32;
@@ -62,7 +63,9 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_W = OFF_K + STAGES * KEY_STAGE_BYTES;
-  static constexpr int OFF_BAR = OFF_W + W_FLOATS * 4;
+  static constexpr int HIST_BINS = 4096;  // decode: first-digit histogram of the scores for the Top-k
+  static constexpr int OFF_HIST = OFF_W + W_FLOATS * 4;
+  static constexpr int OFF_BAR = OFF_HIST + (PAGED ? HIST_BINS * 4 : 0);
   static constexpr int N_BARS = 2 * STAGES + 2 * NBUF + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
@@ -82,6 +85,7 @@ struct Params {
   int32_t max_pages;
   int32_t n_pages;
   int32_t unit_tiles;       // key tiles per CTA
+  uint32_t* hist;           // paged only, or null: [n_q][4096] counts of f32_key(score) >> 20, added to
   int* status;
   uint64_t wait_ns;
 };
@@ -146,6 +150,9 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
+  if (PAGED && p.hist)
+    for (int i = threadIdx.x; i < C::HIST_BINS; i += C::THREADS) hist_s[i] = 0u;
   // per-(query, head) weights, folded with the query scale
   if (warp >= 2) {
     const int et = threadIdx.x - 64;
@@ -302,7 +309,10 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
           float acc = a2.x + a2.y;
           if (FP8) acc *= sk;
           if (PAGED) {
-            if (s_abs < len) p.scores[static_cast<int64_t>(b) * p.ld + s_abs] = acc;
+            if (s_abs < len) {
+              p.scores[static_cast<int64_t>(b) * p.ld + s_abs] = acc;
+              if (p.hist) atomicAdd(&hist_s[f32_key(acc) >> 20], 1u);
+            }
           } else {
             const int32_t row = r0 + g * C::NQ + qq;
             if (row < p.n_q && s_abs <= static_cast<int64_t>(p.q_pos0) + row && s_abs < p.n_tokens)
@@ -344,6 +354,11 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (PAGED && p.hist) {  // this CTA's counts into the sequence's histogram
+    uint32_t* g = p.hist + static_cast<int64_t>(b) * C::HIST_BINS;
+    for (int i = threadIdx.x; i < C::HIST_BINS; i += C::THREADS)
+      if (hist_s[i]) atomicAdd(&g[i], hist_s[i]);
+  }
   if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 

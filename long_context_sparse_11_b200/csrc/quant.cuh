@@ -43,13 +43,11 @@ namespace dsa {
 // out of range is skipped and flagged in the status word.
 constexpr int CACHE_WRITE_MAX_CHUNKS = 5;  // ceil(576 / 4 / 32)
 
-__global__ void __launch_bounds__(256) cache_write_e4m3_kernel(
-    const uint16_t* __restrict__ x, int32_t n_rows, int32_t dim, const int32_t* __restrict__ seq,
-    const int32_t* __restrict__ pos, const int32_t* __restrict__ block_table, int32_t batch, int32_t max_pages,
-    int32_t n_pages, uint8_t* __restrict__ pool, float* __restrict__ pool_scale, int* status) {
-  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (r >= n_rows) return;
+__device__ __forceinline__ void cache_write_row(const uint16_t* __restrict__ x, int64_t r, int lane, int32_t dim,
+                                                const int32_t* __restrict__ seq, const int32_t* __restrict__ pos,
+                                                const int32_t* __restrict__ block_table, int32_t batch,
+                                                int32_t max_pages, int32_t n_pages, uint8_t* __restrict__ pool,
+                                                float* __restrict__ pool_scale, int* status) {
   const int32_t b = seq ? seq[r] : static_cast<int32_t>(r);
   const int32_t t = pos[r];
   int32_t page = -1;
@@ -92,6 +90,38 @@ __global__ void __launch_bounds__(256) cache_write_e4m3_kernel(
     }
   }
   if (lane == 0) pool_scale[slot] = s;
+}
+
+__global__ void __launch_bounds__(256) cache_write_e4m3_kernel(
+    const uint16_t* __restrict__ x, int32_t n_rows, int32_t dim, const int32_t* __restrict__ seq,
+    const int32_t* __restrict__ pos, const int32_t* __restrict__ block_table, int32_t batch, int32_t max_pages,
+    int32_t n_pages, uint8_t* __restrict__ pool, float* __restrict__ pool_scale, int* status) {
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (r >= n_rows) return;
+  cache_write_row(x, r, threadIdx.x & 31, dim, seq, pos, block_table, batch, max_pages, n_pages, pool, pool_scale,
+                  status);
+}
+
+// The same write for up to CACHE_WRITE_MAX_POOLS pools in one launch (every layer's latent pool
+// and every Full layer's key pool of a decode step: the same sequences, positions and pages).
+// blockIdx.y selects the pool.
+constexpr int CACHE_WRITE_MAX_POOLS = 128;
+struct CacheWritePools {
+  const uint16_t* x[CACHE_WRITE_MAX_POOLS];
+  uint8_t* pool[CACHE_WRITE_MAX_POOLS];
+  float* scale[CACHE_WRITE_MAX_POOLS];
+  int32_t dim[CACHE_WRITE_MAX_POOLS];
+};
+
+__global__ void __launch_bounds__(256) cache_write_e4m3_pools_kernel(
+    const __grid_constant__ CacheWritePools pools, int32_t n_rows, const int32_t* __restrict__ seq,
+    const int32_t* __restrict__ pos, const int32_t* __restrict__ block_table, int32_t batch, int32_t max_pages,
+    int32_t n_pages, int* status) {
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (r >= n_rows) return;
+  const int i = blockIdx.y;
+  cache_write_row(pools.x[i], r, threadIdx.x & 31, pools.dim[i], seq, pos, block_table, batch, max_pages, n_pages,
+                  pools.pool[i], pools.scale[i], status);
 }
 
 }  // namespace dsa

@@ -15,7 +15,8 @@ and latent caches).  One IndexShare group step, on every rank:
 Only candidates (2 x k values per index row per rank) and partial results cross ranks; no cache
 row moves.  The step is written once, as a generator that yields at each collective, and run by
 one of two drivers: ``run_distributed`` (torch.distributed all-gather, NCCL on GPUs) or
-``run_emulated`` (all ranks in one process, one after another; what a single GPU can test).
+``run_emulated`` (all ranks in one process, one after another; what a single GPU can test); the
+drivers also run other step generators (``cp.group_step``).
 ``DeviceOps`` supplies the steps from the CUDA library; any object with the same five methods
 can stand in for it.
 """
@@ -64,9 +65,10 @@ def group_step(ops, s: RankSlice):
     return idx_global, results
 
 
-def run_distributed(ops, s: RankSlice, all_gather):
-    """Drive one rank's step; all_gather(t) -> [G, *t.shape] stack in rank order (collective)."""
-    gen = group_step(ops, s)
+def run_distributed(ops, s, all_gather, step=None):
+    """Drive one rank's step (``group_step`` unless another step generator is given);
+    all_gather(t) -> [G, *t.shape] stack in rank order (collective)."""
+    gen = (step or group_step)(ops, s)
     try:
         t = next(gen)
         while True:
@@ -75,10 +77,10 @@ def run_distributed(ops, s: RankSlice, all_gather):
         return stop.value
 
 
-def run_emulated(ops, slices, stack):
+def run_emulated(ops, slices, stack, step=None):
     """Drive every rank's step in one process, in lock step at each collective; stack(list) ->
     [G, ...].  Returns each rank's result."""
-    gens = [group_step(ops, s) for s in slices]
+    gens = [(step or group_step)(ops, s) for s in slices]
     pending = [next(g) for g in gens]
     results = [None] * len(gens)
     while any(r is None for r in results):

@@ -172,3 +172,12 @@ def test_product_path_never_imports_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in txt.lower(), f
+
+
+def test_projection_arguments_are_checked(lib):
+    # widths that are not multiples of 64, and a missing workspace, fail before any launch
+    assert lib.dsa_indexer_project(16, 16, 16, 16, 16, 16, 4, 100, 6144, 16, 16, 16, 16, 1 << 20, None) == \
+        B.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_indexer_project(16, 16, 16, 16, 16, 16, 4, 2048, 6144, 16, 16, 16, 16, 8, None) == \
+        B.DSA_ERR_WORKSPACE
+    assert lib.dsa_mla_latent(16, 16, 16, 16, 4, 6144, 0.5, 16, 16, 1 << 20, None) == B.DSA_ERR_INVALID_ARG

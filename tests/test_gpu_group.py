@@ -299,3 +299,27 @@ def test_paged_attention_query_values_within_and_beyond_f16_range():
         dsa.sync_status()
     assert e.value.status == dsa.binding.DSA_ERR_RANGE
     dsa.sync_status()                                           # the status word was cleared
+
+
+def test_decode_group_long_rows_take_the_fused_histogram():
+    """Rows longer than 32,768 keys in a small batch take the segmented Top-k, whose first-digit
+    histogram the paged indexer builds in its epilogue: the sets still match the oracle's."""
+    spec = DecodeSpec("h", batch=3, ctx_lo=33000, ctx_hi=70000, rows_per_seq=2, k=2048, n_layers=1, seed=15)
+    inp = make_decode(spec)
+    g, _, _ = _paged_group(spec, inp)
+    out, _ = g.forward()
+    dsa.sync_status()
+    idx = g.idx.cpu().numpy()
+    q8, sq = O.quantize_e4m3_rows(inp["q_idx"], 128)
+    qv = O.e4m3_to_f64(q8) * sq.reshape(-1, 32, 1)
+    for b in range(spec.batch):
+        n = int(inp["ctx"][b])
+        assert n > 32768
+        kk = O.paged_rows(inp["idx_keys"], inp["idx_key_scale"], inp["block_table"][b], n)
+        sc = O.indexer_scores(qv[b:b + 1], inp["w"][b:b + 1], kk, [n])[0]
+        check_topk_sets(idx[b], sc, n, spec.k)
+    o = O.bf16_to_f64(bf16_host(out[0]))
+    kv = O.paged_rows(inp["KV"][0], inp["KV_scale"][0], inp["block_table"][1], int(inp["ctx"][1]))
+    ref, _ = O.sparse_mla_row(O.bf16_to_f64(inp["Q"][0][2]), kv, idx[1], inp["softmax_scale"])
+    ma, rel = attn_errors(o[2], ref)
+    assert ma <= 2e-2 and rel <= 5e-3

@@ -77,3 +77,20 @@ def test_mla_latent_rows_and_query_rope():
     assert np.array_equal(gq[:, :, :512], q[:, :, :512])
     rq = O.rope_query(O.bf16_to_f64(q), qpos)
     _close_bf16(O.bf16_to_f64(gq[:, :, 512:]), rq[:, :, 512:])
+
+
+@pytest.mark.parametrize("q_rank,hidden", [(64, 64), (192, 320)])
+def test_indexer_projections_small_widths(q_rank, hidden):
+    """The projections at the smallest widths the library takes (one or a few 64-wide K blocks)."""
+    T = 70
+    cq, x = _bf16(81, (T, q_rank)), _bf16(82, (T, hidden))
+    Wq, Wkw = _bf16(83, (4096, q_rank), q_rank ** -0.5), _bf16(84, (160, hidden), hidden ** -0.5)
+    gamma, beta = np.full(128, 1.25, dtype=np.float32), np.full(128, -0.5, dtype=np.float32)
+    q, k, w = dsa.indexer_project(bf16_dev(cq), bf16_dev(x), bf16_dev(Wq), bf16_dev(Wkw), f32_dev(gamma), f32_dev(beta))
+    dsa.sync_status()
+    rq, rk, rw = O.indexer_projections(O.bf16_to_f64(cq), O.bf16_to_f64(x), O.bf16_to_f64(Wq),
+                                       O.bf16_to_f64(Wkw[:128]), O.bf16_to_f64(Wkw[128:]), gamma, beta)
+    _close_bf16(O.bf16_to_f64(bf16_host(q)), rq)
+    _close_bf16(O.bf16_to_f64(bf16_host(k)), rk)
+    assert np.max(np.abs(w.cpu().numpy() - rw)) <= 1e-4 * np.max(np.abs(rw))
+

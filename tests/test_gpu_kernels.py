@@ -131,6 +131,29 @@ def test_cache_write_e4m3_bit_exact():
     assert np.array_equal(pool_d.cpu().numpy(), ref_pool) and np.array_equal(scale_d.cpu().numpy(), ref_scale)
 
 
+def test_cache_write_pools_in_one_launch_equals_the_oracle():
+    """A decode step's writes into two latent pools and one key pool through one launch: every pool
+    bit-exact with the oracle's write of its own rows."""
+    spec = DecodeSpec("c", batch=4, ctx_lo=100, ctx_hi=900, rows_per_seq=1, k=8, n_layers=2, seed=14)
+    inp = make_decode(spec)
+    bt, ctx = inp["block_table"], inp["ctx"]
+    pos = (ctx - 1).astype(np.int32)                                # the current token of each sequence
+    targets = [(576, inp["KV"][0], inp["KV_scale"][0]), (576, inp["KV"][1], inp["KV_scale"][1]),
+               (128, inp["idx_keys"], inp["idx_key_scale"])]
+    writes, refs = [], []
+    for i, (dim, pool, scale) in enumerate(targets):
+        bits = bf16_bits_np(normal_np(50 + i, 0, 4 * dim).reshape(4, dim) * 2.0)
+        refs.append(O.cache_write_e4m3(pool, scale, bt, bits, np.arange(4), pos))
+        writes.append((bf16_dev(bits), u8_dev(pool), f32_dev(scale)))
+    before = dsa.load().dsa_launch_count()
+    dsa.CacheWriteBatch(writes, i32_dev(pos), i32_dev(bt))()
+    assert dsa.load().dsa_launch_count() == before + 1
+    dsa.sync_status()
+    for (x, pool_d, scale_d), (ref_pool, ref_scale) in zip(writes, refs):
+        assert np.array_equal(pool_d.cpu().numpy(), ref_pool)
+        assert np.array_equal(scale_d.cpu().numpy(), ref_scale)
+
+
 # ----------------------------------------------------------------------------- a4
 
 
