@@ -13,7 +13,7 @@ Default (``all``): the headline line is causal prefill of 131,072 tokens with th
 (the largest single-GPU prefill workload), timed over exactly K steps; the same process then
 measures the other workloads (512-token tiny prefill, 32K bf16 prefill, batch-32 decode with 4
 MTP draft rows and without, 1M-token 78-layer decode) and reports each under ``workloads``, each
-timed over at least one second of steps so that the clock sampler sees it.
+timed over at least two seconds of steps so that the clock sampler sees it.
 
 One JSON line is printed by rank 0.  Multi-GPU (torchrun): every rank runs its own independent
 problem (weak scaling, no collective on the data path); the time is the max over ranks of the
@@ -58,7 +58,7 @@ def parse(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     p.add_argument("--ref-seconds", type=float, default=150.0, help="reference arm total budget")
     p.add_argument("--seq-len", type=int, default=None, help="override L of a prefill workload (profiling)")
-    p.add_argument("--min-timed-s", type=float, default=1.0,
+    p.add_argument("--min-timed-s", type=float, default=2.0,
                    help="least timed seconds of each workload under 'workloads' (clock samples)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-sub", action="store_true", help="headline workload only")
@@ -344,6 +344,7 @@ class ClockSampler:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(1.0)   # nvidia-smi's start-up: the first sample should fall inside the timed region
         except OSError:
             self.proc = None
         return self

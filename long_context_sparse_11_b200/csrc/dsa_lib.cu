@@ -10,6 +10,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -18,6 +19,7 @@
 #include "gemm.cuh"
 #include "indexer.cuh"
 #include "mla.cuh"
+#include "mla_db.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 #include "splitn.cuh"
@@ -79,7 +81,9 @@ struct DeviceState {
   bool ready = false;
   int sms = 148;
   int* status = nullptr;
-  int paged_indexer_ctas_per_sm = 1;  // resident CTAs of the paged indexer kernel per SM
+  // bf16 latent table: the single-tile kernel (default), or the half-tile double-buffered one
+  // when DSA_MLA_DENSE=halves is set in the environment when the device is first used
+  bool mla_db = false;
 };
 
 DeviceState g_dev[64];
@@ -114,12 +118,6 @@ dsa_status device_state(DeviceState** out) {
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             idx::Cfg<true, true>::SMEM_BYTES),
                        "smem attr"));
-    DSA_TRY(cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.paged_indexer_ctas_per_sm,
-                                                                     idx::indexer_kernel<true, true>,
-                                                                     idx::Cfg<true, true>::THREADS,
-                                                                     idx::Cfg<true, true>::SMEM_BYTES),
-                       "occupancy"));
-    d.paged_indexer_ctas_per_sm = std::max(1, d.paged_indexer_ctas_per_sm);
     DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<false, false>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES),
                        "smem attr"));
@@ -132,6 +130,13 @@ dsa_status device_state(DeviceState** out) {
     DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<true, true>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES),
                        "smem attr"));
+    DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::db::sparse_mla_db_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, mla::db::SMEM_BYTES),
+                       "smem attr"));
+    {
+      const char* e = std::getenv("DSA_MLA_DENSE");
+      d.mla_db = e && std::strcmp(e, "halves") == 0;
+    }
     DSA_TRY(cuda_check(cudaFuncSetAttribute(gemm::gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             gemm::SMEM_BYTES),
                        "smem attr"));
@@ -239,16 +244,10 @@ dsa_status launch_indexer(const void* q, int32_t q_dtype, const float* q_scale, 
     DSA_TRY(make_map(&mk, keys->data, false, 128, static_cast<uint64_t>(keys->n_tokens), 128, 128, 64));
     const int64_t max_len = static_cast<int64_t>(keys->max_pages) * DSA_PAGE;
     const int64_t tiles = (max_len + idx::BLOCK_KEYS - 1) / idx::BLOCK_KEYS;
-    // few long sequences: cut each into units so that the CTAs fill the GPU's resident slots a
-    // whole number of times (a partial last wave left a 1M-token sequence at 0.47 of HBM); many
-    // sequences keep 32-tile units, fine-grained enough to balance their different lengths
+    // few long sequences: shorter units, so that the grid still covers the SMs several times over
+    // (units sized to fill exactly one wave of resident CTAs measured slower on a 1M-token sequence)
     int32_t unit = idx::UNIT_TILES;
-    const int64_t slots = static_cast<int64_t>(ds->paged_indexer_ctas_per_sm) * ds->sms;
-    if (static_cast<int64_t>(n_q) * ((tiles + unit - 1) / unit) < 4 * slots) {
-      const int64_t waves = std::max<int64_t>(1, (static_cast<int64_t>(n_q) * tiles + 64 * slots - 1) / (64 * slots));
-      unit = static_cast<int32_t>(std::max<int64_t>(4, (static_cast<int64_t>(n_q) * tiles + waves * slots - 1) /
-                                                       (waves * slots)));
-    }
+    while (unit > 4 && static_cast<int64_t>(n_q) * ((tiles + unit - 1) / unit) < 4LL * ds->sms) unit /= 2;
     p.unit_tiles = unit;
     dim3 grid(static_cast<unsigned>((tiles + unit - 1) / unit), static_cast<unsigned>(n_q));
     using C = idx::Cfg<true, true>;
@@ -433,7 +432,9 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
   const unsigned grid = sk.on ? static_cast<unsigned>(sk.grid)
                               : static_cast<unsigned>(std::min<int64_t>(static_cast<int64_t>(n_q) * p.n_split,
                                                                         static_cast<int64_t>(ds->sms)));
-  if (paged && sk.on) {
+  if (!paged && !sk.on && ds->mla_db) {
+    mla::db::sparse_mla_db_kernel<<<grid, mla::THREADS, mla::db::SMEM_BYTES, st>>>(p);
+  } else if (paged && sk.on) {
     mla::sparse_mla_kernel<true, true><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
   } else if (paged) {
     mla::sparse_mla_kernel<true, false><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);

@@ -292,7 +292,9 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
         // head sum of one query from registers: ReLU, per-head weight, packed FMA on head pairs
         auto score = [&](const uint32_t (&x)[32], int qq) {
           const float4* wv = reinterpret_cast<const float4*>(w_s + (g * C::NQ + qq) * 32);
-          float2 a2 = make_float2(0.f, 0.f);
+          // two independent chains of packed FMAs (heads 0-1, 4-5, ... and 2-3, 6-7, ...), so
+          // that consecutive FMAs of one query do not wait on each other
+          float2 a2 = make_float2(0.f, 0.f), b2 = make_float2(0.f, 0.f);
 #pragma unroll
           for (int h4 = 0; h4 < 8; ++h4) {
             const float4 ww = wv[h4];
@@ -304,9 +306,9 @@ __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
             }
             // packed fp32 FMA on head pairs (the compiler's own pairing of the operands)
             a2 = __ffma2_rn(make_float2(ww.x, ww.y), make_float2(r[0], r[1]), a2);
-            a2 = __ffma2_rn(make_float2(ww.z, ww.w), make_float2(r[2], r[3]), a2);
+            b2 = __ffma2_rn(make_float2(ww.z, ww.w), make_float2(r[2], r[3]), b2);
           }
-          float acc = a2.x + a2.y;
+          float acc = (a2.x + a2.y) + (b2.x + b2.y);
           if (FP8) acc *= sk;
           if (PAGED) {
             if (s_abs < len) {

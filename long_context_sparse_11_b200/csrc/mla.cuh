@@ -759,11 +759,17 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
 
 // Combine split-KV partials: one CTA of 128 threads per (row, head), 4 dims per thread.  Equal
 // splits: n_split slots per row.  Stream-K (grid > 0): the row's fragments came from CTAs
-// sk_owner(first tile) .. sk_owner(last tile); a row inside one CTA was written directly.
+// sk_owner(first tile) .. sk_owner(last tile); a row inside one CTA was written directly.  A row
+// has at most MAX_SLOTS fragments (one per 128-key tile of k <= 2048); their weights are formed
+// once in shared memory and the partial rows are read with every load in flight at once (the
+// reads, not the arithmetic, set the time of this short kernel).
+constexpr int MAX_SLOTS = 16;
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part_o,
                                                       const float* __restrict__ part_ml, int32_t n_split,
                                                       uint16_t* __restrict__ out, float* __restrict__ lse,
                                                       int32_t tiles_per_row, int64_t sk_tiles, int32_t sk_grid) {
+  __shared__ float wgt_s[MAX_SLOTS];
+  __shared__ float tot_s[2];  // max (log2 units), sum of weighted row sums
   const int32_t row = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
   int32_t n_slots = n_split;
   if (sk_grid > 0) {
@@ -772,25 +778,40 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
                                    sk_owner(g0, sk_tiles, sk_grid) + 1);
     if (n_slots == 1) return;
   }
-  float M = -INFINITY;
-  for (int s = 0; s < n_slots; ++s) {
-    const int64_t pr = static_cast<int64_t>(row) * n_split + s;
-    if (part_ml[pr * 128 + 64 + h] > 0.f) M = fmaxf(M, part_ml[pr * 128 + h]);
+  n_slots = min(n_slots, MAX_SLOTS);
+  if (t < 32) {
+    const int64_t pr = static_cast<int64_t>(row) * n_split + t;
+    const bool live = t < n_slots && part_ml[pr * 128 + 64 + h] > 0.f;
+    const float m = live ? part_ml[pr * 128 + h] : -INFINITY;
+    const float l = live ? part_ml[pr * 128 + 64 + h] : 0.f;
+    float M = m;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float w = live ? exp2f(m - M) : 0.f;
+    float L = w * l;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    if (t < MAX_SLOTS) wgt_s[t] = w;
+    if (t == 0) {
+      tot_s[0] = M;
+      tot_s[1] = L;
+    }
   }
-  float L = 0.f;
+  __syncthreads();
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < n_slots; ++s) {
-    const int64_t pr = static_cast<int64_t>(row) * n_split + s;
-    const float l = part_ml[pr * 128 + 64 + h];
-    if (!(l > 0.f)) continue;
-    const float wgt = exp2f(part_ml[pr * 128 + h] - M);
-    L = fmaf(wgt, l, L);
-    const float4 o = *reinterpret_cast<const float4*>(part_o + (pr * 64 + h) * 512 + 4 * t);
-    acc.x = fmaf(wgt, o.x, acc.x);
-    acc.y = fmaf(wgt, o.y, acc.y);
-    acc.z = fmaf(wgt, o.z, acc.z);
-    acc.w = fmaf(wgt, o.w, acc.w);
+#pragma unroll
+  for (int s = 0; s < MAX_SLOTS; ++s) {
+    const float w = wgt_s[s];
+    if (s < n_slots && w > 0.f) {
+      const int64_t pr = static_cast<int64_t>(row) * n_split + s;
+      const float4 o = *reinterpret_cast<const float4*>(part_o + (pr * 64 + h) * 512 + 4 * t);
+      acc.x = fmaf(w, o.x, acc.x);
+      acc.y = fmaf(w, o.y, acc.y);
+      acc.z = fmaf(w, o.z, acc.z);
+      acc.w = fmaf(w, o.w, acc.w);
+    }
   }
+  const float M = tot_s[0], L = tot_s[1];
   const float inv = L > 0.f ? 1.f / L : 0.f;
   const __nv_bfloat162 a = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
   const __nv_bfloat162 b = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
