@@ -10,7 +10,6 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -19,7 +18,6 @@
 #include "gemm.cuh"
 #include "indexer.cuh"
 #include "mla.cuh"
-#include "mla_db.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 #include "splitn.cuh"
@@ -81,9 +79,6 @@ struct DeviceState {
   bool ready = false;
   int sms = 148;
   int* status = nullptr;
-  // bf16 latent table: the single-tile kernel (default), or the half-tile double-buffered one
-  // when DSA_MLA_DENSE=halves is set in the environment when the device is first used
-  bool mla_db = false;
 };
 
 DeviceState g_dev[64];
@@ -130,13 +125,6 @@ dsa_status device_state(DeviceState** out) {
     DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::sparse_mla_kernel<true, true>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, mla::SMEM_BYTES),
                        "smem attr"));
-    DSA_TRY(cuda_check(cudaFuncSetAttribute(mla::db::sparse_mla_db_kernel,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize, mla::db::SMEM_BYTES),
-                       "smem attr"));
-    {
-      const char* e = std::getenv("DSA_MLA_DENSE");
-      d.mla_db = e && std::strcmp(e, "halves") == 0;
-    }
     DSA_TRY(cuda_check(cudaFuncSetAttribute(gemm::gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             gemm::SMEM_BYTES),
                        "smem attr"));
@@ -432,9 +420,7 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
   const unsigned grid = sk.on ? static_cast<unsigned>(sk.grid)
                               : static_cast<unsigned>(std::min<int64_t>(static_cast<int64_t>(n_q) * p.n_split,
                                                                         static_cast<int64_t>(ds->sms)));
-  if (!paged && !sk.on && ds->mla_db) {
-    mla::db::sparse_mla_db_kernel<<<grid, mla::THREADS, mla::db::SMEM_BYTES, st>>>(p);
-  } else if (paged && sk.on) {
+  if (paged && sk.on) {
     mla::sparse_mla_kernel<true, true><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
   } else if (paged) {
     mla::sparse_mla_kernel<true, false><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);

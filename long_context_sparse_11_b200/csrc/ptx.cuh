@@ -46,18 +46,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking probe of the phase with the given parity (never suspends the thread): for a
-// thread that polls several barriers in turn.
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait for the phase with the given parity, giving up after limit_ns (or when another
 // role of the CTA already gave up).  On time-out: sets *abort (shared) and the device
 // status word, returns false.  Every spin in this library goes through here.
@@ -223,16 +211,6 @@ __host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c) {
       "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),                                                          \
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),      \
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])                       \
-      : "memory")
-
-// 16 lanes x 8 columns, twice: threads 0-15 read lanes base..base+15 at columns col..col+7,
-// threads 16-31 the same lanes at columns col+8..col+15 (the row layout of an M = 64 accumulator).
-#define DSA_TMEM_LD_16X2_X8(taddr, r)                                                                         \
-  asm volatile(                                                                                               \
-      "tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], 8;\n\t"                      \
-      "tcgen05.wait::ld.sync.aligned;"                                                                        \
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])        \
-      : "r"(taddr)                                                                                            \
       : "memory")
 
 // TMEM load without the wait, and a wait that names the destination registers so that no use
