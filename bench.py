@@ -42,10 +42,10 @@ SUB_WORKLOADS = ["tiny_prefill", "prefill_32k", "decode_b32_mtp4", "decode_b32_d
 ALL_WORKLOADS = ["tiny_prefill", "prefill_32k", "prefill_128k_fp8", "decode_b32_mtp4", "decode_b32_d0",
                  "decode_b32_mtp4_verify", "decode_1m_mtp5"]
 
-# sparse_mla_kernel<bf16>, L=8,192 prefill launch (8,192 query rows): ncu measured 672.8 MB read
-# + 510.4 MB written = 144,436 B per query row (queries 73,728 B in, outputs 65,536 B out, the
+# sparse_mla_kernel<bf16>, L=8,192 prefill launch (8,192 query rows): ncu measured 672.9 MB read
+# + 505.9 MB written = 143,893 B per query row (queries 73,728 B in, outputs 65,536 B out, the
 # rest index rows and the latent rows' first touch).
-MLA_DRAM_BYTES_PER_ROW_BF16 = (672.798720e6 + 510.417920e6) / 8192
+MLA_DRAM_BYTES_PER_ROW_BF16 = (672.903936e6 + 505.879296e6) / 8192
 
 
 def parse(argv=None):
@@ -396,6 +396,31 @@ def measured_peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+def fp8_dense_peak(dev):
+    """Dense e4m3 GEMM throughput on this GPU: the library FP8 GEMM (cuBLASLt through
+    torch._scaled_mm, 8192^3, bf16 out), best of 10 after warm-up; None if unavailable."""
+    import torch
+    try:
+        n = 8192
+        a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        for _ in range(3):
+            torch._scaled_mm(a, b, one, one, out_dtype=torch.bfloat16)
+        best = float("inf")
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(10):
+            e0.record()
+            torch._scaled_mm(a, b, one, one, out_dtype=torch.bfloat16)
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        del a, b
+        return 2.0 * n ** 3 / (best / 1e3) / 1e12
+    except Exception:
+        return None
+
+
 # ----------------------------------------------------------------------------- CPU oracle sample
 
 
@@ -648,6 +673,13 @@ def measure(name, args, ws, rank, local, headline):
                                    "peak": round(ia_peak, 1), "frac": round(ia_tf / ia_peak, 4),
                                    "peak_source": f"{peak_kind} bf16 dense (burst)" +
                                    (" x 2 (fp8 / bf16 nominal)" if wl.spec.indexer_fp8 else "")}
+        if wl.spec.indexer_fp8:
+            f8 = fp8_dense_peak(dev)
+            if f8:
+                phases["indexer_alone"].update({
+                    "fp8_gemm_tflops": round(f8, 1), "frac_of_fp8_gemm": round(ia_tf / f8, 4),
+                    "fp8_gemm_source": "library e4m3 GEMM on this GPU (torch._scaled_mm, 8192^3, bf16 out, "
+                                       "best of 10)"})
         proj = input_projections(wl.spec.L, dev, stream)
         for v in proj.values():
             v.update({"peak": bf16_peak, "frac": round(v["tflops"] / bf16_peak, 4),

@@ -131,10 +131,6 @@ dsa_status device_state(DeviceState** out) {
     DSA_TRY(cuda_check(cudaFuncSetAttribute(topk::topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             static_cast<int>(sizeof(topk::Smem))),
                        "smem attr"));
-    DSA_TRY(cuda_check(cudaFuncSetAttribute(topk::topk_seg_resolve_kernel,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            static_cast<int>(sizeof(topk::Smem))),
-                       "smem attr"));
     d.ready = true;
   }
   *out = &d;
@@ -326,9 +322,7 @@ dsa_status launch_topk(const float* scores, int64_t ld, int32_t n_rows, const in
   }
   topk::topk_seg_filter_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k,
                                                                    pl.seg_len, sw, idx_out);
-  topk::topk_seg_resolve_kernel<<<n_rows, topk::THREADS, sizeof(topk::Smem), st>>>(scores, ld, row_len,
-                                                                                  causal_len0, cap, k, sw, idx_out);
-  count_launch(2);
+  count_launch();
   return cuda_check(cudaGetLastError(), "topk launch");
 }
 
@@ -1087,8 +1081,6 @@ extern "C" dsa_status dsa_topk_no_alloc(const float* scores, int64_t ld, int32_t
                                                                  sw);
   topk::topk_seg_filter_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k,
                                                                    seg_len, sw, idx_out);
-  topk::topk_seg_resolve_kernel<<<n_rows, topk::THREADS, sizeof(topk::Smem), st>>>(scores, ld, row_len, causal_len0,
-                                                                                  cap, k, sw, idx_out);
-  count_launch(3);
+  count_launch(2);
   return cuda_check(cudaGetLastError(), "no-alloc top-k launch");
 }

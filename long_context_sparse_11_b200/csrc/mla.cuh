@@ -359,7 +359,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
   // once PV of the previous tile has released it.  bf16: cp.async, and the hardware arrives on
   // the sub-tile's "full" barrier when this thread's copies have landed (the thread never waits
   // for them; the MMA issuer fences the async proxy after the barrier).
-  constexpr int MAXC = (1024 + NG - 1) / NG;
+  // 16-byte chunks per sub-tile: 1,024 for the bf16 cache (128 keys x 8), 512 parts for FP8 (128 x 4)
+  constexpr int MAXC = ((PAGED ? 512 : 1024) + NG - 1) / NG;
   struct Plan {
     const uint8_t* src[MAXC];
     uint32_t nb[MAXC], dst[MAXC];
@@ -456,34 +457,28 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
           cp_async16(base + OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7), qsrc + h * 1152 + ch * 16, 16);
         }
       } else {
-        // batches of QB loads in flight before the first conversion; values that f16 cannot hold
-        // (|q| >= 65520 rounds to infinity) are reported through the status word
-        constexpr int QPER = (QCH + GA_THREADS - 1) / GA_THREADS, QB = 3;  // chunks c >= QCH are skipped
+        // every chunk copied at once (one memory latency per row), then converted bf16 -> f16 in
+        // place by the thread that copied it; values that f16 cannot hold (|q| >= 65520 rounds to
+        // infinity) are reported through the status word
+        for (int c = gq; c < QCH; c += GA_THREADS) {
+          const int h = c / 72, ch = c % 72;
+          cp_async16(base + OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7), qsrc + h * 1152 + ch * 16, 16);
+        }
+        cp_async_wait_all();
         bool out_of_range = false;
-        for (int b0 = 0; b0 < QPER; b0 += QB) {
-          uint4 raw[QB];
+        for (int c = gq; c < QCH; c += GA_THREADS) {
+          const int h = c / 72, ch = c % 72;
+          uint4* chunk = reinterpret_cast<uint4*>(smem + OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7));
+          const uint4 raw = *chunk;
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t o[4];
 #pragma unroll
-          for (int j = 0; j < QB; ++j) {
-            const int c = gq + (b0 + j) * GA_THREADS;
-            raw[j] = c < QCH ? __ldg(reinterpret_cast<const uint4*>(qsrc + (c / 72) * 1152 + (c % 72) * 16))
-                             : make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < 4; ++i) {
+            const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+            out_of_range |= fmaxf(fabsf(lo), fabsf(hi)) >= 65520.f;
+            o[i] = pack_pair(lo, hi, true);
           }
-#pragma unroll
-          for (int j = 0; j < QB; ++j) {
-            const int c = gq + (b0 + j) * GA_THREADS;
-            if (c >= QCH) continue;
-            const int h = c / 72, ch = c % 72;
-            const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
-            uint32_t o[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
-              out_of_range |= fmaxf(fabsf(lo), fabsf(hi)) >= 65520.f;
-              o[i] = pack_pair(lo, hi, true);
-            }
-            *reinterpret_cast<uint4*>(smem + OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7)) =
-                make_uint4(o[0], o[1], o[2], o[3]);
-          }
+          *chunk = make_uint4(o[0], o[1], o[2], o[3]);
         }
         if (out_of_range) atomicOr(p.status, DEVERR_RANGE);
       }
@@ -583,6 +578,18 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         Plan next_plan;  // indices of the next tile, loaded while this tile's softmax runs
         if (SM_GATHER && t + 1 < it.n_tiles) next_plan = prepare(it, t + 1, threadIdx.x);
         const float kscale = PAGED ? (valid ? p.kv_scale[prow] : 0.f) : 1.f;
+        if (PAGED && t + 1 < it.n_tiles) {
+          // FP8 cache rows live in HBM (the pools are far larger than L2): start bringing the next
+          // tile's rows into L2 now (before waiting for S^T, which takes longer than the index
+          // loads), so that its loads after this softmax wait for L2, not HBM.  The thread that
+          // owns the first 16 values of a key fetches that key's five 128-byte lines (a 576-byte
+          // row starts at offset 0 or 64 of a line).  A tile has 512 parts and at least as many
+          // gathering threads, so a thread has one part at most.
+          static_assert(!PAGED || MAXC == 1, "one FP8 part per thread");
+          if (next_plan.nb[0] && (next_plan.dst[0] & 3u) == 0u)
+#pragma unroll
+            for (int l = 0; l < 5; ++l) prefetch_l2(next_plan.src[0] + 128 * l);
+        }
         {
           const bool got = mbar_wait(bar(B_SFULL), par, abort_flag, p.status, p.wait_ns);
           fail = __any_sync(0xffffffffu, fail || !got);   // warp-uniform: the TMEM load is collective

@@ -11,8 +11,9 @@
 // Row mode (one CTA per row): the row is read twice from global memory (histogram of the
 // first digit, then emit / collect the threshold bin into shared memory); later digits
 // run on the shared-memory candidates.  Segmented mode (few long rows): several CTAs per
-// row build the first-digit histogram and emit / collect in parallel through a global
-// workspace; one CTA per row then resolves the remaining digits.
+// row build the first-digit histogram (or the paged indexer builds it in its epilogue), then
+// several CTAs per row emit / collect in parallel through a global workspace, and the last of
+// them to finish resolves the remaining digits.
 #pragma once
 #include "ptx.cuh"
 
@@ -100,9 +101,18 @@ struct CandSrc {
   __device__ __forceinline__ int32_t index(int32_t i) const { return idx[i]; }
 };
 
+struct CandSrcL2 {  // candidates written by other CTAs of the grid: read at L2, past this SM's L1
+  const uint32_t* keys;
+  const int32_t* idx;
+  int32_t n;
+  __device__ __forceinline__ int32_t size() const { return n; }
+  __device__ __forceinline__ uint64_t comp(int32_t i) const { return composite(__ldcg(keys + i), __ldcg(idx + i)); }
+  __device__ __forceinline__ int32_t index(int32_t i) const { return __ldcg(idx + i); }
+};
+
 // Walk digits lvl0..5 over `src`, emitting into out[0..k) through the shared counter.
-template <int NT, class Src>
-__device__ void walk_digits(const Src& src, int lvl0, uint64_t pfx, uint64_t pmask, uint32_t k_rem, Smem& sm,
+template <int NT, class Src, class S>
+__device__ void walk_digits(const Src& src, int lvl0, uint64_t pfx, uint64_t pmask, uint32_t k_rem, S& sm,
                             int32_t* out, int32_t kmax) {
   const int t = threadIdx.x;
   for (int lvl = lvl0; lvl < 6 && k_rem > 0; ++lvl) {
@@ -262,6 +272,23 @@ __global__ void __launch_bounds__(SEG_THREADS) topk_seg_hist_kernel(const float*
     if (hist[b]) atomicAdd(&g[b], hist[b]);
 }
 
+// Filter and resolve in one launch.  Every CTA of a row emits the elements above the threshold
+// bin of the row's first-digit histogram and collects the threshold bin's elements into the row's
+// global candidate list; the last CTA of the row to finish (counted on counters[2], after a
+// device-scope fence of each CTA's writes) then resolves the remaining digits over those candidates.
+struct FilterSmem {
+  static constexpr int SEL_BUF = 2048, CAND_BUF = 1024;
+  uint32_t hist[BINS];
+  uint32_t warp_sum[32];
+  int32_t out_cnt;
+  uint32_t sel_bin, sel_above, sel_eq;
+  int32_t s_sel[SEL_BUF];
+  uint32_t s_ckey[CAND_BUF];
+  int32_t s_cidx[CAND_BUF];
+  int32_t s_cnt[2], s_base[2];
+  int32_t last;
+};
+
 __global__ void __launch_bounds__(SEG_THREADS) topk_seg_filter_kernel(const float* __restrict__ scores, int64_t ld,
                                                                       const int32_t* __restrict__ row_len,
                                                                       int64_t causal_len0, int64_t cap, int32_t k,
@@ -270,31 +297,31 @@ __global__ void __launch_bounds__(SEG_THREADS) topk_seg_filter_kernel(const floa
   // The segment's selections and threshold-bin candidates are gathered in shared memory and
   // placed in the row's arrays with one global reservation each per CTA: a per-element atomic
   // on the row's counter serialises about k same-address atomics per row.
-  constexpr int SEL_BUF = 2048, CAND_BUF = 1024;
-  __shared__ uint32_t hist[BINS];
-  __shared__ uint32_t warp_sum[32];
-  __shared__ uint32_t sel[3];
-  __shared__ int32_t s_sel[SEL_BUF];
-  __shared__ uint32_t s_ckey[CAND_BUF];
-  __shared__ int32_t s_cidx[CAND_BUF];
-  __shared__ int32_t s_cnt[2], s_base[2];
+  __shared__ FilterSmem sm;
+  constexpr int SEL_BUF = FilterSmem::SEL_BUF, CAND_BUF = FilterSmem::CAND_BUF;
   const int32_t r = blockIdx.y;
+  const int t = threadIdx.x;
   const int32_t n = row_length(r, row_len, causal_len0, cap);
-  if (n <= k) return;
+  int32_t* out = idx_out + static_cast<int64_t>(r) * k;
+  if (n <= k) {  // every candidate is selected, the rest is padding
+    if (blockIdx.x == 0)
+      for (int32_t i = t; i < k; i += SEG_THREADS) out[i] = i < n ? i : -1;
+    return;
+  }
   const int32_t beg = blockIdx.x * seg_len;
   if (beg >= n) return;
+  const int32_t n_segs = (n + seg_len - 1) / seg_len;  // CTAs of this row that reach the end
   const int32_t end = min(n, beg + seg_len);
-  const int t = threadIdx.x;
   const uint32_t* g = ws.hist + static_cast<int64_t>(r) * BINS;
-  for (int b = t; b < BINS; b += SEG_THREADS) hist[b] = g[b];
-  if (t == 0) s_cnt[0] = s_cnt[1] = 0;
+  for (int b = t; b < BINS; b += SEG_THREADS) sm.hist[b] = g[b];
+  if (t == 0) sm.s_cnt[0] = sm.s_cnt[1] = 0;
   __syncthreads();
-  find_threshold<SEG_THREADS>(hist, static_cast<uint32_t>(k), warp_sum, &sel[0], &sel[1], &sel[2]);
-  const uint32_t T = sel[0], above = sel[1], eq = sel[2];
+  find_threshold<SEG_THREADS>(sm.hist, static_cast<uint32_t>(k), sm.warp_sum, &sm.sel_bin, &sm.sel_above,
+                              &sm.sel_eq);
+  const uint32_t T = sm.sel_bin, above = sm.sel_above, eq = sm.sel_eq;
   const bool take_eq = (eq == static_cast<uint32_t>(k) - above);
   const bool collect = !take_eq && eq <= static_cast<uint32_t>(ws.gcap);
   const float* row = scores + static_cast<int64_t>(r) * ld;
-  int32_t* out = idx_out + static_cast<int64_t>(r) * k;
   int32_t* cnt = ws.counters + static_cast<int64_t>(r) * 4;
   uint32_t* ck = ws.cand_key + static_cast<int64_t>(r) * ws.gcap;
   int32_t* ci = ws.cand_idx + static_cast<int64_t>(r) * ws.gcap;
@@ -302,18 +329,18 @@ __global__ void __launch_bounds__(SEG_THREADS) topk_seg_filter_kernel(const floa
     const uint32_t key = f32_key(f);
     const uint32_t d = key >> 20;
     if (d > T || (take_eq && d == T)) {
-      const int32_t p = atomicAdd(&s_cnt[0], 1);
+      const int32_t p = atomicAdd(&sm.s_cnt[0], 1);
       if (p < SEL_BUF) {
-        s_sel[p] = i;
+        sm.s_sel[p] = i;
       } else {  // overflow (a segment holding more than SEL_BUF selections): place directly
         const int32_t pos = atomicAdd(&cnt[0], 1);
         if (pos < k) out[pos] = i;
       }
     } else if (collect && d == T) {
-      const int32_t p = atomicAdd(&s_cnt[1], 1);
+      const int32_t p = atomicAdd(&sm.s_cnt[1], 1);
       if (p < CAND_BUF) {
-        s_ckey[p] = key;
-        s_cidx[p] = i;
+        sm.s_ckey[p] = key;
+        sm.s_cidx[p] = i;
       } else {
         const int32_t c = atomicAdd(&cnt[1], 1);
         if (c < ws.gcap) {
@@ -349,69 +376,41 @@ __global__ void __launch_bounds__(SEG_THREADS) topk_seg_filter_kernel(const floa
   }
   for (int32_t u = end4 + t; u < end; u += SEG_THREADS) visit(row[u], u);
   __syncthreads();
-  const int32_t n_sel = min(s_cnt[0], SEL_BUF), n_cand = min(s_cnt[1], CAND_BUF);
+  const int32_t n_sel = min(sm.s_cnt[0], SEL_BUF), n_cand = min(sm.s_cnt[1], CAND_BUF);
   if (t == 0) {
-    s_base[0] = n_sel > 0 ? atomicAdd(&cnt[0], n_sel) : 0;
-    s_base[1] = n_cand > 0 ? atomicAdd(&cnt[1], n_cand) : 0;
+    sm.s_base[0] = n_sel > 0 ? atomicAdd(&cnt[0], n_sel) : 0;
+    sm.s_base[1] = n_cand > 0 ? atomicAdd(&cnt[1], n_cand) : 0;
   }
   __syncthreads();
   for (int32_t j = t; j < n_sel; j += SEG_THREADS) {
-    const int32_t pos = s_base[0] + j;
-    if (pos < k) out[pos] = s_sel[j];
+    const int32_t pos = sm.s_base[0] + j;
+    if (pos < k) out[pos] = sm.s_sel[j];
   }
   for (int32_t j = t; j < n_cand; j += SEG_THREADS) {
-    const int32_t c = s_base[1] + j;
+    const int32_t c = sm.s_base[1] + j;
     if (c < ws.gcap) {
-      ck[c] = s_ckey[j];
-      ci[c] = s_cidx[j];
+      ck[c] = sm.s_ckey[j];
+      ci[c] = sm.s_cidx[j];
     }
   }
-}
-
-__global__ void __launch_bounds__(THREADS) topk_seg_resolve_kernel(const float* __restrict__ scores, int64_t ld,
-                                                                   const int32_t* __restrict__ row_len,
-                                                                   int64_t causal_len0, int64_t cap, int32_t k,
-                                                                   SegWs ws, int32_t* __restrict__ idx_out) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
-  const int32_t r = blockIdx.x;
-  const int t = threadIdx.x;
-  const int32_t n = row_length(r, row_len, causal_len0, cap);
-  int32_t* out = idx_out + static_cast<int64_t>(r) * k;
-  if (n <= k) {
-    for (int32_t i = t; i < k; i += THREADS) out[i] = i < n ? i : -1;
-    return;
-  }
-  const uint32_t* g = ws.hist + static_cast<int64_t>(r) * BINS;
-  for (int b = t; b < BINS; b += THREADS) sm.hist[b] = g[b];
+  // ---- the row's last CTA resolves the threshold bin
+  __threadfence();
   __syncthreads();
-  find_threshold<THREADS>(sm.hist, static_cast<uint32_t>(k), sm.warp_sum, &sm.sel_bin, &sm.sel_above, &sm.sel_eq);
-  const uint32_t T = sm.sel_bin, above = sm.sel_above, eq = sm.sel_eq;
+  if (t == 0) sm.last = atomicAdd(&cnt[2], 1) == n_segs - 1;
+  __syncthreads();
+  if (!sm.last || take_eq) return;  // take_eq: the filter emitted the whole Top-k
+  __threadfence();
   const uint32_t k_rem = static_cast<uint32_t>(k) - above;
-  if (eq == k_rem) return;  // the filter pass emitted everything
   if (t == 0) sm.out_cnt = static_cast<int32_t>(above);
-  const int32_t* cnt = ws.counters + static_cast<int64_t>(r) * 4;
   const uint64_t pfx = static_cast<uint64_t>(T) << 52;
   const uint64_t pmask = static_cast<uint64_t>(0xFFF) << 52;
-  const uint32_t* ck = ws.cand_key + static_cast<int64_t>(r) * ws.gcap;
-  const int32_t* ci = ws.cand_idx + static_cast<int64_t>(r) * ws.gcap;
-  if (eq <= static_cast<uint32_t>(CAND_CAP)) {
-    const int32_t c = min(cnt[1], CAND_CAP);
-    for (int32_t i = t; i < c; i += THREADS) {
-      sm.cand_key[i] = ck[i];
-      sm.cand_idx[i] = ci[i];
-    }
-    __syncthreads();
-    CandSrc src{sm.cand_key, sm.cand_idx, c};
-    walk_digits<THREADS>(src, 1, pfx, pmask, k_rem, sm, out, k);
-  } else if (eq <= static_cast<uint32_t>(ws.gcap)) {
-    __syncthreads();
-    CandSrc src{ck, ci, min(cnt[1], ws.gcap)};
-    walk_digits<THREADS>(src, 1, pfx, pmask, k_rem, sm, out, k);
+  __syncthreads();
+  if (collect) {
+    CandSrcL2 src{ck, ci, min(__ldcg(&cnt[1]), ws.gcap)};
+    walk_digits<SEG_THREADS>(src, 1, pfx, pmask, k_rem, sm, out, k);
   } else {
-    __syncthreads();
-    RowSrc src{scores + static_cast<int64_t>(r) * ld, n};
-    walk_digits<THREADS>(src, 1, pfx, pmask, k_rem, sm, out, k);
+    RowSrc src{row, n};
+    walk_digits<SEG_THREADS>(src, 1, pfx, pmask, k_rem, sm, out, k);
   }
 }
 

@@ -197,6 +197,27 @@ def test_topk_segmented_crowded_threshold_bin():
         assert set(got[r]) == set(ref), r
 
 
+@pytest.mark.parametrize("k", [2048, 100, 1])
+def test_topk_long_rows_in_row_mode(k):
+    """Row mode (one CTA per row) on rows of 16K-32K candidates with awkward value patterns:
+    heavy ties, all-equal scores, values rising along the row, and outliers on a regular
+    stride.  Each row's set equals the oracle's."""
+    rows, L = 8, 32768
+    s = normal_np(91, 0, rows * L).reshape(rows, L)
+    s[1] = np.round(s[1] * 8) / 8                        # heavy ties
+    s[2] = 1.0                                            # all equal: the band holds every score
+    s[3] = np.arange(L) / L + 1e-3 * s[3]                 # rising: the top-k sits at the end
+    s[4, ::64] += 50.0                                    # outliers on a stride of 64
+    s[5, 8::64] += 50.0                                   # the same, shifted
+    s = s.astype(np.float32)
+    lens = np.array([L, L, L, L, L, L, 16384, 20001], dtype=np.int32)
+    out = dsa.topk(f32_dev(s), k, row_len=i32_dev(lens), max_len=L)
+    got = out.cpu().numpy()
+    for r in range(rows):
+        ref = O.topk_row(s[r].astype(np.float64), int(lens[r]), k)
+        assert set(got[r]) == set(ref), r
+
+
 def test_topk_causal_lengths():
     rows, L, k = 64, 600, 256
     s = normal_np(3, 0, rows * L).reshape(rows, L).astype(np.float32)
