@@ -578,18 +578,6 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         Plan next_plan;  // indices of the next tile, loaded while this tile's softmax runs
         if (SM_GATHER && t + 1 < it.n_tiles) next_plan = prepare(it, t + 1, threadIdx.x);
         const float kscale = PAGED ? (valid ? p.kv_scale[prow] : 0.f) : 1.f;
-        if (PAGED && t + 1 < it.n_tiles) {
-          // FP8 cache rows live in HBM (the pools are far larger than L2): start bringing the next
-          // tile's rows into L2 now (before waiting for S^T, which takes longer than the index
-          // loads), so that its loads after this softmax wait for L2, not HBM.  The thread that
-          // owns the first 16 values of a key fetches that key's five 128-byte lines (a 576-byte
-          // row starts at offset 0 or 64 of a line).  A tile has 512 parts and at least as many
-          // gathering threads, so a thread has one part at most.
-          static_assert(!PAGED || MAXC == 1, "one FP8 part per thread");
-          if (next_plan.nb[0] && (next_plan.dst[0] & 3u) == 0u)
-#pragma unroll
-            for (int l = 0; l < 5; ++l) prefetch_l2(next_plan.src[0] + 128 * l);
-        }
         {
           const bool got = mbar_wait(bar(B_SFULL), par, abort_flag, p.status, p.wait_ns);
           fail = __any_sync(0xffffffffu, fail || !got);   // warp-uniform: the TMEM load is collective

@@ -92,10 +92,6 @@ __device__ __forceinline__ void fence_async_smem() {
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
-// Bring the global-memory line holding p into L2 (no register result, no wait).
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
-}
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 // Arrive on the mbarrier once all of this thread's earlier cp.async copies have landed; the
 // thread itself does not wait (the arrival counts against the barrier's expected count).
