@@ -428,8 +428,10 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
           e4m3x16_to_f16(raw[d], o0, o1);
           *reinterpret_cast<uint4*>(smem + OFF_KV + d * SUB_KV + sw128_off(key, 2 * part)) = o0;
           *reinterpret_cast<uint4*>(smem + OFF_KV + d * SUB_KV + sw128_off(key, 2 * part + 1)) = o1;
-          // the MMA issuer fences the async proxy once after the barrier (as for cp.async data)
-          if (last) mbar_arrive(bar(B_FULL + d));
+          if (last) {
+            fence_async_smem();
+            mbar_arrive(bar(B_FULL + d));
+          }
         }
         if (!free_ok) return false;
       }
