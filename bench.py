@@ -516,6 +516,7 @@ def measure(name, args, ws, rank, local, headline):
     lib = dsa.load()
     dev = torch.device("cuda", local)
     spec, cfg = workload_config(name, args.seq_len if headline else None)
+    mem0 = torch.cuda.memory_allocated(dev)
     wl = Workload(spec, name, dev)
     counts = wl.counts
     stream = torch.cuda.current_stream()
@@ -693,20 +694,31 @@ def measure(name, args, ws, rank, local, headline):
             "how": "both timed with CUDA events, L2 flushed before each; the 4 independent layers are 4 "
                    "one-layer group calls that each run their own a1-a4 and a6"}
 
+    per_set = torch.cuda.memory_allocated(dev) - mem0   # one set of inputs, outputs and workspace
+
     def make_twin():
         """A second set of device inputs/outputs (the same seeded data), so that one step's upload
-        can run while the previous step computes; None when the GPU has no room for it."""
-        free, _ = torch.cuda.mem_get_info()
-        if free < 1.25 * torch.cuda.memory_allocated() + (4 << 30):
+        can run while the previous step computes; None when the GPU has no room for it (the free
+        device memory plus what the caching allocator holds unused, against one set's bytes and a
+        3 GiB margin; an allocation that still fails falls back to one set)."""
+        free, _ = torch.cuda.mem_get_info(dev)
+        avail = free + torch.cuda.memory_reserved(dev) - torch.cuda.memory_allocated(dev)
+        if avail < per_set + (3 << 30):
             return None
-        wl2 = Workload(spec, name, dev)
-        wl2.forward()
-        g2 = None
-        if graph is not None:
-            g2 = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g2):
-                wl2.forward()
-        torch.cuda.synchronize()
+        try:
+            wl2 = Workload(spec, name, dev)
+            wl2.forward()
+            g2 = None
+            if graph is not None:
+                g2 = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g2):
+                    wl2.forward()
+            torch.cuda.synchronize()
+        except torch.cuda.OutOfMemoryError:
+            wl2 = g2 = None
+            gc.collect()
+            torch.cuda.empty_cache()
+            return None
         return wl2, (g2.replay if g2 is not None else wl2.forward), g2
 
     e2e = None
