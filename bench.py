@@ -144,7 +144,7 @@ def algorithmic_counts(spec, ctx=None):
         pairs = L * (L + 1) // 2
         sel = sum(min(k, t + 1) for t in range(L))
         return {"tokens": L, "indexer_flops": 8192.0 * pairs, "mla_flops_per_layer": 139264.0 * sel,
-                "mla_rows": L, "indexer_bytes": None}
+                "mla_rows": L, "indexer_bytes": None, "mla_gather_bytes_per_layer": 1152.0 * sel}
     import numpy as np
     ctx = np.asarray(ctx)
     R = spec.rows_per_seq
@@ -641,6 +641,10 @@ def measure(name, args, ws, rank, local, headline):
     phases = {"indexer_topk_ms": round(idx_avg, 4), "mla_ms_per_layer": round(mla_avg, 4),
               "indexer_topk_tflops": round(counts["indexer_flops"] / (idx_avg / 1e3) / 1e12, 1),
               "groups_per_step": n_groups}
+    if counts.get("mla_gather_bytes_per_layer"):
+        # context for the sparse MLA roofline: the selected 1,152-byte latent rows it gathers from
+        # L2 into shared memory per launch, as an aggregate rate (the kernel's limiter, not HBM)
+        phases["mla_gather_tbs"] = round(counts["mla_gather_bytes_per_layer"] / (mla_avg / 1e3) / 1e12, 2)
     roofline = mla_roof
     if counts.get("indexer_bytes"):
         gbs = counts["indexer_bytes"] / (idx_avg / 1e3) / 1e9
