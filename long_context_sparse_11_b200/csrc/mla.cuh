@@ -774,11 +774,23 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
     if (n_slots == 1) return;
   }
   n_slots = min(n_slots, MAX_SLOTS);
+  const int64_t pr0 = static_cast<int64_t>(row) * n_split;
+  auto load_o = [&](int s) {
+    return *reinterpret_cast<const float4*>(part_o + ((pr0 + s) * 64 + h) * 512 + 4 * t);
+  };
+  // the first slots' partial rows in flight before their weights are known, with the row sums and
+  // maxima: one memory latency instead of three in a chain (row sum, max, then the rows)
+  constexpr int EARLY = 4;
+  float4 o[EARLY];
+#pragma unroll
+  for (int s = 0; s < EARLY; ++s) o[s] = s < n_slots ? load_o(s) : make_float4(0.f, 0.f, 0.f, 0.f);
   if (t < 32) {
-    const int64_t pr = static_cast<int64_t>(row) * n_split + t;
-    const bool live = t < n_slots && part_ml[pr * 128 + 64 + h] > 0.f;
-    const float m = live ? part_ml[pr * 128 + h] : -INFINITY;
-    const float l = live ? part_ml[pr * 128 + 64 + h] : 0.f;
+    const int64_t pr = pr0 + t;
+    const float l_raw = t < n_slots ? part_ml[pr * 128 + 64 + h] : 0.f;
+    const float m_raw = t < n_slots ? part_ml[pr * 128 + h] : -INFINITY;
+    const bool live = l_raw > 0.f;
+    const float m = live ? m_raw : -INFINITY;
+    const float l = live ? l_raw : 0.f;
     float M = m;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
@@ -794,17 +806,24 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
   }
   __syncthreads();
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  // a slot without keys (weight 0) holds no written row: it never enters acc
+  auto add = [&](float w, const float4& v) {
+    acc.x = fmaf(w, v.x, acc.x);
+    acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z);
+    acc.w = fmaf(w, v.w, acc.w);
+  };
 #pragma unroll
-  for (int s = 0; s < MAX_SLOTS; ++s) {
-    const float w = wgt_s[s];
-    if (s < n_slots && w > 0.f) {
-      const int64_t pr = static_cast<int64_t>(row) * n_split + s;
-      const float4 o = *reinterpret_cast<const float4*>(part_o + (pr * 64 + h) * 512 + 4 * t);
-      acc.x = fmaf(w, o.x, acc.x);
-      acc.y = fmaf(w, o.y, acc.y);
-      acc.z = fmaf(w, o.z, acc.z);
-      acc.w = fmaf(w, o.w, acc.w);
-    }
+  for (int s = 0; s < EARLY; ++s)
+    if (s < n_slots && wgt_s[s] > 0.f) add(wgt_s[s], o[s]);
+  // rows cut into more slots (few rows over many CTAs): the rest in batches of EARLY, loads first
+  for (int s0 = EARLY; s0 < n_slots; s0 += EARLY) {
+#pragma unroll
+    for (int u = 0; u < EARLY; ++u)
+      o[u] = s0 + u < n_slots && wgt_s[s0 + u] > 0.f ? load_o(s0 + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < EARLY; ++u)
+      if (s0 + u < n_slots && wgt_s[s0 + u] > 0.f) add(wgt_s[s0 + u], o[u]);
   }
   const float M = tot_s[0], L = tot_s[1];
   const float inv = L > 0.f ? 1.f / L : 0.f;
