@@ -426,8 +426,15 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
   count_launch();
   DSA_TRY(cuda_check(cudaGetLastError(), "sparse MLA launch"));
   if (p.n_split > 1) {
-    mla::combine_kernel<<<dim3(n_q, 64), 128, 0, st>>>(p.part_o, p.part_ml, p.n_split, p.out, p.lse,
-                                                      sk.tiles_per_row, sk.tiles, sk.on ? sk.grid : 0);
+    // rows cut into more than 4 slots, few enough that all (row, head) blocks run in one wave
+    // even at the occupancy of the all-slots variant (6 blocks per SM): every slot in flight
+    const bool all_slots = p.n_split > 4 && static_cast<int64_t>(n_q) * 64 <= 6LL * ds->sms;
+    if (all_slots)
+      mla::combine_kernel<mla::MAX_SLOTS><<<dim3(n_q, 64), 128, 0, st>>>(
+          p.part_o, p.part_ml, p.n_split, p.out, p.lse, sk.tiles_per_row, sk.tiles, sk.on ? sk.grid : 0);
+    else
+      mla::combine_kernel<4><<<dim3(n_q, 64), 128, 0, st>>>(p.part_o, p.part_ml, p.n_split, p.out, p.lse,
+                                                           sk.tiles_per_row, sk.tiles, sk.on ? sk.grid : 0);
     count_launch();
     DSA_TRY(cuda_check(cudaGetLastError(), "combine launch"));
   }

@@ -759,6 +759,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
 // once in shared memory and the partial rows are read with every load in flight at once (the
 // reads, not the arithmetic, set the time of this short kernel).
 constexpr int MAX_SLOTS = 16;
+// EARLY: slots whose rows are loaded before the weights.  4 keeps the registers low enough for a
+// grid of many waves; MAX_SLOTS (every slot at once) suits a grid of few rows cut into many slots.
+template <int EARLY>
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part_o,
                                                       const float* __restrict__ part_ml, int32_t n_split,
                                                       uint16_t* __restrict__ out, float* __restrict__ lse,
@@ -780,7 +783,6 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
   };
   // the first slots' partial rows in flight before their weights are known, with the row sums and
   // maxima: one memory latency instead of three in a chain (row sum, max, then the rows)
-  constexpr int EARLY = 4;
   float4 o[EARLY];
 #pragma unroll
   for (int s = 0; s < EARLY; ++s) o[s] = s < n_slots ? load_o(s) : make_float4(0.f, 0.f, 0.f, 0.f);

@@ -389,7 +389,7 @@ def test_sparse_mla_k_covers_history_is_dense():
         assert ma <= 2e-2 and rl <= 5e-3, (t, ma, rl)
 
 
-@pytest.mark.parametrize("B,R,k", [(2, 3, 256), (3, 5, 2048), (40, 1, 512)])
+@pytest.mark.parametrize("B,R,k", [(2, 3, 256), (3, 5, 2048), (40, 1, 512), (2, 3, 2048)])
 def test_sparse_mla_paged_fp8_mtp(B, R, k):
     spec = DecodeSpec("t", batch=B, ctx_lo=100, ctx_hi=5000, rows_per_seq=R, k=k, n_layers=1, seed=50 + B)
     inp = make_decode(spec)
