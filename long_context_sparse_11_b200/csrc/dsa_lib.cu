@@ -10,9 +10,11 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "../../include/dsa.h"
 #include "gemm.cuh"
@@ -47,6 +49,33 @@ int64_t g_wait_ns = 2000000000LL;
 std::atomic<int64_t> g_launches{0};
 
 void count_launch(int n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// Programmatic dependent launch for the kernels of a group (each starts with grid_dependency_sync):
+// a kernel's launch overlaps the completion of the previous kernel of the stream, which matters for
+// decode steps of a few hundred short kernels.  DSA_PDL=0 in the environment launches them plainly
+// (same results, for timing the difference).
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("DSA_PDL");
+    return e == nullptr || std::atoi(e) != 0;
+  }();
+  return on;
+}
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  // a failed launch is left for the caller's cudaGetLastError, like a <<<>>> launch
+  (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 void trace(void** ev, int i, cudaStream_t st) {
   if (ev && ev[i]) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st);
@@ -235,7 +264,7 @@ dsa_status launch_indexer(const void* q, int32_t q_dtype, const float* q_scale, 
     p.unit_tiles = unit;
     dim3 grid(static_cast<unsigned>((tiles + unit - 1) / unit), static_cast<unsigned>(n_q));
     using C = idx::Cfg<true, true>;
-    idx::indexer_kernel<true, true><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, p);
+    launch_pdl(idx::indexer_kernel<true, true>, grid, C::THREADS, C::SMEM_BYTES, st, mq, mk, p);
     count_launch();
   } else {
     const int64_t max_len = std::min<int64_t>(static_cast<int64_t>(q_pos0) + n_q, keys->n_tokens);
@@ -248,7 +277,7 @@ dsa_status launch_indexer(const void* q, int32_t q_dtype, const float* q_scale, 
                        static_cast<uint64_t>(keys->row_stride), 128, 128));
       dim3 grid(static_cast<unsigned>((tiles + idx::UNIT_TILES - 1) / idx::UNIT_TILES),
                 static_cast<unsigned>((n_q + 15) / 16));
-      idx::indexer_kernel<true, false><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, p);
+      launch_pdl(idx::indexer_kernel<true, false>, grid, C::THREADS, C::SMEM_BYTES, st, mq, mk, p);
       count_launch();
     } else {
       using C = idx::Cfg<false, false>;
@@ -257,7 +286,7 @@ dsa_status launch_indexer(const void* q, int32_t q_dtype, const float* q_scale, 
                        static_cast<uint64_t>(keys->row_stride) * 2, 64, 128));
       dim3 grid(static_cast<unsigned>((tiles + idx::UNIT_TILES - 1) / idx::UNIT_TILES),
                 static_cast<unsigned>((n_q + 15) / 16));
-      idx::indexer_kernel<false, false><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, p);
+      launch_pdl(idx::indexer_kernel<false, false>, grid, C::THREADS, C::SMEM_BYTES, st, mq, mk, p);
       count_launch();
     }
   }
@@ -298,7 +327,7 @@ dsa_status launch_topk(const float* scores, int64_t ld, int32_t n_rows, const in
   const int64_t cap = std::min(ld, max_len);
   const TopkPlan pl = plan_topk(n_rows, cap, k, ds->sms);
   if (!pl.segmented) {
-    topk::topk_row_kernel<<<n_rows, topk::THREADS, sizeof(topk::Smem), st>>>(scores, ld, n_rows, row_len,
+    launch_pdl(topk::topk_row_kernel, n_rows, topk::THREADS, sizeof(topk::Smem), st, scores, ld, n_rows, row_len,
                                                                              causal_len0, cap, k, idx_out);
     count_launch();
     return cuda_check(cudaGetLastError(), "topk launch");
@@ -316,11 +345,11 @@ dsa_status launch_topk(const float* scores, int64_t ld, int32_t n_rows, const in
   dim3 grid(pl.segs, n_rows);
   if (!hist_ready) {
     DSA_TRY(cuda_check(cudaMemsetAsync(ws, 0, head, st), "topk workspace clear"));
-    topk::topk_seg_hist_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k,
+    launch_pdl(topk::topk_seg_hist_kernel, grid, topk::SEG_THREADS, 0, st, scores, ld, row_len, causal_len0, cap, k,
                                                                    pl.seg_len, sw);
     count_launch();
   }
-  topk::topk_seg_filter_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k,
+  launch_pdl(topk::topk_seg_filter_kernel, grid, topk::SEG_THREADS, 0, st, scores, ld, row_len, causal_len0, cap, k,
                                                                    pl.seg_len, sw, idx_out);
   count_launch();
   return cuda_check(cudaGetLastError(), "topk launch");
@@ -415,13 +444,13 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
                               : static_cast<unsigned>(std::min<int64_t>(static_cast<int64_t>(n_q) * p.n_split,
                                                                         static_cast<int64_t>(ds->sms)));
   if (paged && sk.on) {
-    mla::sparse_mla_kernel<true, true><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
+    launch_pdl(mla::sparse_mla_kernel<true, true>, grid, mla::THREADS, mla::SMEM_BYTES, st, p);
   } else if (paged) {
-    mla::sparse_mla_kernel<true, false><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
+    launch_pdl(mla::sparse_mla_kernel<true, false>, grid, mla::THREADS, mla::SMEM_BYTES, st, p);
   } else if (sk.on) {
-    mla::sparse_mla_kernel<false, true><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
+    launch_pdl(mla::sparse_mla_kernel<false, true>, grid, mla::THREADS, mla::SMEM_BYTES, st, p);
   } else {
-    mla::sparse_mla_kernel<false, false><<<grid, mla::THREADS, mla::SMEM_BYTES, st>>>(p);
+    launch_pdl(mla::sparse_mla_kernel<false, false>, grid, mla::THREADS, mla::SMEM_BYTES, st, p);
   }
   count_launch();
   DSA_TRY(cuda_check(cudaGetLastError(), "sparse MLA launch"));
@@ -430,10 +459,10 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
     // even at the occupancy of the all-slots variant (6 blocks per SM): every slot in flight
     const bool all_slots = p.n_split > 4 && static_cast<int64_t>(n_q) * 64 <= 6LL * ds->sms;
     if (all_slots)
-      mla::combine_kernel<mla::MAX_SLOTS><<<dim3(n_q, 64), 128, 0, st>>>(
+      launch_pdl(mla::combine_kernel<mla::MAX_SLOTS>, dim3(n_q, 64), 128, 0, st,
           p.part_o, p.part_ml, p.n_split, p.out, p.lse, sk.tiles_per_row, sk.tiles, sk.on ? sk.grid : 0);
     else
-      mla::combine_kernel<4><<<dim3(n_q, 64), 128, 0, st>>>(p.part_o, p.part_ml, p.n_split, p.out, p.lse,
+      launch_pdl(mla::combine_kernel<4>, dim3(n_q, 64), 128, 0, st, p.part_o, p.part_ml, p.n_split, p.out, p.lse,
                                                            sk.tiles_per_row, sk.tiles, sk.on ? sk.grid : 0);
     count_launch();
     DSA_TRY(cuda_check(cudaGetLastError(), "combine launch"));
@@ -667,7 +696,7 @@ dsa_status dsa_quant_e4m3(const void* x_bf16, int64_t n_vec, int32_t vec_len, ui
   DSA_TRY(device_state(&ds));
   const int64_t blocks = (n_vec + 7) / 8;
   if (blocks > INT32_MAX) return fail(DSA_ERR_INVALID_ARG, "n_vec too large");
-  quant_e4m3_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  launch_pdl(quant_e4m3_kernel, static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream),
       static_cast<const uint16_t*>(x_bf16), n_vec, codes, scale);
   count_launch();
   return cuda_check(cudaGetLastError(), "quant launch");
@@ -685,7 +714,7 @@ dsa_status dsa_cache_write_e4m3(const void* x_bf16, int32_t n_rows, int32_t dim,
   DeviceState* ds = nullptr;
   DSA_TRY(device_state(&ds));
   const int64_t blocks = (static_cast<int64_t>(n_rows) + 7) / 8;
-  cache_write_e4m3_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  launch_pdl(cache_write_e4m3_kernel, static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream),
       static_cast<const uint16_t*>(x_bf16), n_rows, dim, seq, pos, block_table, batch, max_pages, n_pages, pool,
       pool_scale, ds->status);
   count_launch();
@@ -716,7 +745,7 @@ dsa_status dsa_cache_write_e4m3_pools(int32_t n_pools, const void* const* x_bf16
   DeviceState* ds = nullptr;
   DSA_TRY(device_state(&ds));
   const dim3 grid(static_cast<unsigned>((static_cast<int64_t>(n_rows) + 7) / 8), static_cast<unsigned>(n_pools));
-  cache_write_e4m3_pools_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  launch_pdl(cache_write_e4m3_pools_kernel, grid, 256, 0, static_cast<cudaStream_t>(stream),
       pp, n_rows, seq, pos, block_table, batch, max_pages, n_pages, ds->status);
   count_launch();
   return cuda_check(cudaGetLastError(), "cache write launch");
@@ -1084,9 +1113,9 @@ extern "C" dsa_status dsa_topk_no_alloc(const float* scores, int64_t ld, int32_t
   // the histograms and counters of the previous call must not leak into this one
   DSA_TRY(cuda_check(cudaMemsetAsync(scratch, 0, head, st), "clear top-k scratch"));
   dim3 grid(static_cast<unsigned>(segs), static_cast<unsigned>(n_rows));
-  topk::topk_seg_hist_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k, seg_len,
+  launch_pdl(topk::topk_seg_hist_kernel, grid, topk::SEG_THREADS, 0, st, scores, ld, row_len, causal_len0, cap, k, seg_len,
                                                                  sw);
-  topk::topk_seg_filter_kernel<<<grid, topk::SEG_THREADS, 0, st>>>(scores, ld, row_len, causal_len0, cap, k,
+  launch_pdl(topk::topk_seg_filter_kernel, grid, topk::SEG_THREADS, 0, st, scores, ld, row_len, causal_len0, cap, k,
                                                                    seg_len, sw, idx_out);
   count_launch(2);
   return cuda_check(cudaGetLastError(), "no-alloc top-k launch");

@@ -93,6 +93,7 @@ struct Params {
 template <bool FP8, bool PAGED>
 __global__ void __launch_bounds__(Cfg<FP8, PAGED>::THREADS, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k, Params p) {
+  grid_dependency_sync();
   using C = Cfg<FP8, PAGED>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);

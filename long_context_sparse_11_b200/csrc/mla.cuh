@@ -314,6 +314,7 @@ __device__ __forceinline__ void e4m3x16_to_f16(uint4 raw, uint4& o0, uint4& o1) 
 
 template <bool PAGED, bool SK>
 __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
+  grid_dependency_sync();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -766,6 +767,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
                                                       const float* __restrict__ part_ml, int32_t n_split,
                                                       uint16_t* __restrict__ out, float* __restrict__ lse,
                                                       int32_t tiles_per_row, int64_t sk_tiles, int32_t sk_grid) {
+  grid_dependency_sync();
   __shared__ float wgt_s[MAX_SLOTS];
   __shared__ float tot_s[2];  // max (log2 units), sum of weighted row sums
   const int32_t row = blockIdx.x, h = blockIdx.y, t = threadIdx.x;

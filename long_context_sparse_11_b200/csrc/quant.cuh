@@ -9,6 +9,7 @@ namespace dsa {
 // One warp per 128-element vector; each lane converts 4 consecutive elements.
 __global__ void __launch_bounds__(256) quant_e4m3_kernel(const uint16_t* __restrict__ x, int64_t n_vec,
                                                          uint8_t* __restrict__ codes, float* __restrict__ scale) {
+  grid_dependency_sync();
   const int64_t vec = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (vec >= n_vec) return;
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(256) cache_write_e4m3_kernel(
     const uint16_t* __restrict__ x, int32_t n_rows, int32_t dim, const int32_t* __restrict__ seq,
     const int32_t* __restrict__ pos, const int32_t* __restrict__ block_table, int32_t batch, int32_t max_pages,
     int32_t n_pages, uint8_t* __restrict__ pool, float* __restrict__ pool_scale, int* status) {
+  grid_dependency_sync();
   const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (r >= n_rows) return;
   cache_write_row(x, r, threadIdx.x & 31, dim, seq, pos, block_table, batch, max_pages, n_pages, pool, pool_scale,
@@ -117,6 +119,7 @@ __global__ void __launch_bounds__(256) cache_write_e4m3_pools_kernel(
     const __grid_constant__ CacheWritePools pools, int32_t n_rows, const int32_t* __restrict__ seq,
     const int32_t* __restrict__ pos, const int32_t* __restrict__ block_table, int32_t batch, int32_t max_pages,
     int32_t n_pages, int* status) {
+  grid_dependency_sync();
   const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (r >= n_rows) return;
   const int i = blockIdx.y;

@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(THREADS) topk_row_kernel(const float* __restri
                                                            int32_t n_rows, const int32_t* __restrict__ row_len,
                                                            int64_t causal_len0, int64_t cap, int32_t k,
                                                            int32_t* __restrict__ idx_out) {
+  grid_dependency_sync();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   const int32_t r = blockIdx.x;
@@ -246,6 +247,7 @@ __global__ void __launch_bounds__(SEG_THREADS) topk_seg_hist_kernel(const float*
                                                                     const int32_t* __restrict__ row_len,
                                                                     int64_t causal_len0, int64_t cap, int32_t k,
                                                                     int32_t seg_len, SegWs ws) {
+  grid_dependency_sync();
   __shared__ uint32_t hist[BINS];
   const int32_t r = blockIdx.y;
   const int32_t n = row_length(r, row_len, causal_len0, cap);
@@ -294,6 +296,7 @@ __global__ void __launch_bounds__(SEG_THREADS) topk_seg_filter_kernel(const floa
                                                                       int64_t causal_len0, int64_t cap, int32_t k,
                                                                       int32_t seg_len, SegWs ws,
                                                                       int32_t* __restrict__ idx_out) {
+  grid_dependency_sync();
   // The segment's selections and threshold-bin candidates are gathered in shared memory and
   // placed in the row's arrays with one global reservation each per CTA: a per-element atomic
   // on the row's counter serialises about k same-address atomics per row.
