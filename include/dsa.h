@@ -22,6 +22,11 @@
  *     caller-provided workspace whose size the *_workspace_bytes() calls return.
  *   - `stream` is a cudaStream_t (may be NULL = legacy default stream).  Every call only
  *     enqueues work and returns; results are ready when the stream reaches that point.
+ *     The kernels of the indexer, Top-k, sparse MLA, quantisation and cache-write calls are
+ *     launched with programmatic dependent launch: each may be launched before the previous
+ *     work of the stream has finished, but waits for it before touching memory, so stream
+ *     order holds as for plain launches (also inside a captured CUDA graph).  Setting
+ *     DSA_PDL=0 in the environment before the first call launches them plainly.
  *   - Arguments are validated on the host before anything is launched; a failing check
  *     returns DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED and launches nothing.  The text
  *     of the last failure on the calling thread is returned by dsa_last_error().
