@@ -181,3 +181,24 @@ def test_projection_arguments_are_checked(lib):
     assert lib.dsa_indexer_project(16, 16, 16, 16, 16, 16, 4, 2048, 6144, 16, 16, 16, 16, 8, None) == \
         B.DSA_ERR_WORKSPACE
     assert lib.dsa_mla_latent(16, 16, 16, 16, 4, 6144, 0.5, 16, 16, 1 << 20, None) == B.DSA_ERR_INVALID_ARG
+
+
+def test_every_kernel_launched_with_programmatic_dependency_waits_first():
+    """Kernels launched with programmatic stream serialisation may start before the previous
+    kernel of the stream has finished; each must wait for it (grid_dependency_sync) before its
+    first memory access, or stream order no longer holds.  Checked on the sources: every kernel
+    named in a launch_pdl call opens with that wait."""
+    csrc = os.path.join(ROOT, "long_context_sparse_11_b200", "csrc")
+    lib_src = open(os.path.join(csrc, "dsa_lib.cu")).read()
+    launched = set(re.findall(r"launch_pdl\(\s*(?:\w+::)*(\w+)\s*[<,]", lib_src))
+    assert {"sparse_mla_kernel", "combine_kernel", "indexer_kernel", "topk_seg_filter_kernel"} <= launched
+    bodies = {}
+    for f in os.listdir(csrc):
+        src = open(os.path.join(csrc, f)).read()
+        for m in re.finditer(r"__global__\s+void\s+(?:__launch_bounds__\([^)]*\)\s*)?(\w+)\s*\(", src):
+            brace = src.index("{", m.end())
+            bodies[m.group(1)] = src[brace + 1:brace + 200]
+    for name in sorted(launched):
+        assert name in bodies, name
+        first = bodies[name].strip().split(";")[0].strip()
+        assert first == "grid_dependency_sync()", (name, first)
