@@ -757,11 +757,12 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
 // splits: n_split slots per row.  Stream-K (grid > 0): the row's fragments came from CTAs
 // sk_owner(first tile) .. sk_owner(last tile); a row inside one CTA was written directly.  A row
 // has at most MAX_SLOTS fragments (one per 128-key tile of k <= 2048); their weights are formed
-// once in shared memory and the partial rows are read with every load in flight at once (the
-// reads, not the arithmetic, set the time of this short kernel).
+// once in shared memory by one warp.  The memory latencies, not the arithmetic, set the time of
+// this short kernel, so the first EARLY slots' partial rows are loaded before the weights, together
+// with the row sums and maxima, and any further slots in batches of EARLY with their loads first.
 constexpr int MAX_SLOTS = 16;
-// EARLY: slots whose rows are loaded before the weights.  4 keeps the registers low enough for a
-// grid of many waves; MAX_SLOTS (every slot at once) suits a grid of few rows cut into many slots.
+// EARLY = 4 keeps the registers low (38) for a grid of many waves; EARLY = MAX_SLOTS (80 registers,
+// every slot at once) suits a grid of few rows cut into many slots, which fits in one wave.
 template <int EARLY>
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part_o,
                                                       const float* __restrict__ part_ml, int32_t n_split,
