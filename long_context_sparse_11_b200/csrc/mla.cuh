@@ -504,7 +504,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
       Item it;
       for (int32_t it_n = 0; ok && work_next<SK>(p, wk, it); ++it_n) {
         if (!mbar_wait(bar(B_QFULL), it_n & 1, abort_flag, p.status, p.wait_ns)) break;
-        fence_async_smem();
+        // cp.async (generic proxy) writes -> tcgen05.mma (async proxy) reads.  On the FP8 path the
+        // writing threads fence their own stores before they arrive, so no fence is needed here.
+        if (!PAGED) fence_async_smem();
         tc_fence_after();
         if (it.n_tiles == 0) mma_commit(bar(B_QEMPTY));
         for (int32_t t = 0; t < it.n_tiles && ok; ++t, ++gtile) {
@@ -515,7 +517,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
               ok = false;
               break;
             }
-            fence_async_smem();  // cp.async (generic proxy) writes -> tcgen05.mma (async proxy) reads
+            if (!PAGED) fence_async_smem();  // as after the query barrier
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
