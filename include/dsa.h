@@ -227,7 +227,9 @@ dsa_status dsa_sparse_mla_attn(const void* q, const dsa_cache_view* kv, const in
  *   workspace: at least dsa_group_workspace_bytes(a) bytes of device memory: e4m3 copies of
  *              the indexer inputs (when quantised here), the scores of one chunk of query rows
  *              (rows x causal length <= max(64 MB, 2,048 x longest row x 4 B), at most 1 GB),
- *              the Top-k scratch and the split-KV partials of the attention.
+ *              the Top-k scratch, the split-KV partials of the attention and, when paged
+ *              layers cut every query row over many CTAs (few rows), the f16 copies of those
+ *              layers' q (converted once per call instead of once per CTA).
  * The call allocates nothing and only enqueues kernels and memsets on `stream`, so once a
  * first call has set the device up it may be captured into a CUDA graph and replayed.
  */

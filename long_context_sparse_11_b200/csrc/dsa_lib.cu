@@ -399,9 +399,19 @@ size_t mla_ws_bytes(int32_t n_q, int32_t k, int sms) {
   return static_cast<size_t>(n_q) * s * (64 * 512 * 4 + 128 * 4) + 256;
 }
 
+// A paged group converts its query rows to f16 once, ahead of the attention, when every row is cut
+// over at least 8 CTAs (few rows): each of those CTAs would otherwise convert the same row.  Measured
+// on decode: 6 rows x 16 splits and 32 rows x 8 splits gain; 160 rows (2-3 stream-K fragments per
+// row) convert inside the kernel, where no extra launch or memory traffic is paid.
+bool mla_query_prepass(int32_t n_q, int32_t k, int sms) {
+  const StreamK sk = plan_stream_k(n_q, k, sms);
+  const int32_t cuts = sk.on ? sk.slots : mla_splits(n_q, k, sms);
+  return cuts >= 8;
+}
+
 dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* idx, int32_t n_q, int32_t rpi,
                       int32_t k, float softmax_scale, void* out, float* lse, void* ws, size_t ws_bytes,
-                      cudaStream_t st, int64_t valid0 = -1) {
+                      cudaStream_t st, int64_t valid0 = -1, const void* q16 = nullptr) {
   DeviceState* ds = nullptr;
   DSA_TRY(device_state(&ds));
   if (n_q == 0) return DSA_OK;
@@ -427,6 +437,10 @@ dsa_status launch_mla(const void* q, const dsa_cache_view* kv, const int32_t* id
   p.wait_ns = static_cast<uint64_t>(g_wait_ns);
   p.n_split = mla_splits(n_q, k, ds->sms);
   p.valid0 = valid0;
+  if (paged && q16) {  // rows converted to f16 ahead of this launch
+    p.q = static_cast<const uint16_t*>(q16);
+    p.q_f16 = 1;
+  }
   // few rows whose tiles all count (decode): contiguous tile ranges per CTA instead of equal splits
   const StreamK sk = valid0 < 0 ? plan_stream_k(n_q, k, ds->sms) : StreamK{};
   if (sk.on) {
@@ -506,6 +520,7 @@ struct Chunk {
 struct GroupPlan {
   bool quant_q = false, quant_k = false;
   size_t off_q8 = 0, off_sq = 0, off_k8 = 0, off_sk = 0, off_scores = 0, off_topk = 0, off_mla = 0, total = 0;
+  size_t off_q16 = 0, q16_layer_bytes = 0;  // f16 query rows of the paged layers (when converted ahead)
   std::vector<Chunk> chunks;
   size_t topk_ws = 0;
 };
@@ -574,6 +589,12 @@ dsa_status plan_group(const dsa_group_args* a, int sms, GroupPlan* g) {
   size_t mla_ws = 0;
   const int32_t nq = a->n_idx_rows * a->q_rows_per_idx_row;
   mla_ws = mla_ws_bytes(nq, a->k, sms);
+  int n_paged = 0;
+  for (int l = 0; l < a->n_layers; ++l) n_paged += a->kv[l].block_table != nullptr;
+  if (n_paged > 0 && mla_query_prepass(nq, a->k, sms)) {
+    g->q16_layer_bytes = static_cast<size_t>(nq) * 64 * 576 * 2;
+    g->off_q16 = take(g->q16_layer_bytes * n_paged);
+  }
   g->off_mla = take(mla_ws);
   g->total = off;
   return DSA_OK;
@@ -1029,10 +1050,30 @@ dsa_status indexshare_group_forward(const dsa_group_args* a, dsa_index_handle* h
   // indices computed by this call for a dense causal prefill: row i holds its min(k, q_pos0 + i + 1)
   // valid entries first, so the attention skips the tiles past them
   const int64_t valid0 = (!reuse_only && !a->idx_keys.block_table) ? static_cast<int64_t>(a->q_pos0) + 1 : -1;
+  // paged layers' query rows to f16 in one launch, when the attention cuts every row over many CTAs
+  // (inside layer 0's trace window: it is attention work)
+  const void* q16[DSA_GROUP_MAX_LAYERS] = {};
+  trace(ev, 2, st);
+  if (g.q16_layer_bytes > 0 && nq > 0) {
+    mla::QConvert qc{};
+    int y = 0;
+    for (int l = 0; l < a->n_layers; ++l) {
+      if (!a->kv[l].block_table) continue;
+      qc.src[y] = static_cast<const uint4*>(a->q[l]);
+      qc.dst[y] = reinterpret_cast<uint4*>(ws + g.off_q16 + y * g.q16_layer_bytes);
+      q16[l] = qc.dst[y];
+      ++y;
+    }
+    const int64_t chunks = static_cast<int64_t>(nq) * 64 * 576 / 8;
+    const unsigned gx = static_cast<unsigned>(std::min<int64_t>((chunks + 255) / 256, 2LL * ds->sms));
+    launch_pdl(mla::q_to_f16_kernel, dim3(gx, static_cast<unsigned>(y)), 256, 0, st, qc, chunks, ds->status);
+    count_launch();
+    DSA_TRY(cuda_check(cudaGetLastError(), "query f16 launch"));
+  }
   for (int l = 0; l < a->n_layers; ++l) {
-    trace(ev, 2 + 2 * l, st);
+    if (l > 0) trace(ev, 2 + 2 * l, st);
     DSA_TRY(launch_mla(a->q[l], &a->kv[l], h->idx, nq, a->q_rows_per_idx_row, a->k, a->softmax_scale, a->out[l],
-                       a->lse[l], ws + g.off_mla, g.total - g.off_mla, st, valid0));
+                       a->lse[l], ws + g.off_mla, g.total - g.off_mla, st, valid0, q16[l]));
     trace(ev, 3 + 2 * l, st);
   }
   return DSA_OK;

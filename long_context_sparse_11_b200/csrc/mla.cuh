@@ -88,7 +88,7 @@ constexpr uint32_t TM_S = 256;  // S^T buffers at columns 256, 320
 constexpr int B_QFULL = 0, B_QEMPTY = 1, B_SFULL = 2, B_PFULL = 3, B_PVDONE = 4, B_FULL = 5, B_EMPTY = 14;
 
 struct Params {
-  const uint16_t* q;         // [n_q,64,576] bf16
+  const uint16_t* q;         // [n_q,64,576] bf16, or its f16 copy when q_f16 is set (paged only)
   const uint8_t* kv;         // dense bf16 [n_tokens,row_stride] or paged e4m3 [n_pages,64,576]
   const float* kv_scale;     // paged: [n_pages*64]
   const int32_t* block_table;
@@ -114,6 +114,7 @@ struct Params {
   float scale_log2;          // softmax_scale * log2(e)
   int* status;
   uint64_t wait_ns;
+  int32_t q_f16;             // paged: 1 when q was converted to f16 before the launch (q_to_f16_kernel)
 };
 
 // Max (or sum) over the 32 lanes of a warp for 32 per-lane values; lane l ends with the
@@ -457,6 +458,12 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
           const int h = c / 72, ch = c % 72;
           cp_async16(base + OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7), qsrc + h * 1152 + ch * 16, 16);
         }
+      } else if (p.q_f16) {
+        // rows converted to f16 before the launch: copied as they are
+        for (int c = gq; c < QCH; c += GA_THREADS) {
+          const int h = c / 72, ch = c % 72;
+          cp_async16(base + OFF_Q + (ch >> 3) * SUB_Q + sw128_off(h, ch & 7), qsrc + h * 1152 + ch * 16, 16);
+        }
       } else {
         // every chunk copied at once (one memory latency per row), then converted bf16 -> f16 in
         // place by the thread that copied it; values that f16 cannot hold (|q| >= 65520 rounds to
@@ -483,7 +490,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
         }
         if (out_of_range) atomicOr(p.status, DEVERR_RANGE);
       }
-      if (!PAGED) {
+      if (!PAGED || p.q_f16) {
         cp_async_arrive_noinc(bar(B_QFULL));
       } else {
         fence_async_smem();
@@ -504,9 +511,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
       Item it;
       for (int32_t it_n = 0; ok && work_next<SK>(p, wk, it); ++it_n) {
         if (!mbar_wait(bar(B_QFULL), it_n & 1, abort_flag, p.status, p.wait_ns)) break;
-        // cp.async (generic proxy) writes -> tcgen05.mma (async proxy) reads.  On the FP8 path the
-        // writing threads fence their own stores before they arrive, so no fence is needed here.
-        if (!PAGED) fence_async_smem();
+        // cp.async (generic proxy) writes -> tcgen05.mma (async proxy) reads.  Rows converted in
+        // the kernel were fenced by the threads that stored them, before they arrived.
+        if (!PAGED || p.q_f16) fence_async_smem();
         tc_fence_after();
         if (it.n_tiles == 0) mma_commit(bar(B_QEMPTY));
         for (int32_t t = 0; t < it.n_tiles && ok; ++t, ++gtile) {
@@ -753,6 +760,36 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_mla_kernel(Params p) {
   __syncthreads();
   tc_fence_after();
   if (warp == MMA_WARP) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// The FP8 path multiplies in f16 (exact for e4m3 keys and values).  When a call cuts every query
+// row over many CTAs, each of them would convert the same row from bf16 to f16, so the rows of
+// all of a group's layers are converted here once, in one launch (blockIdx.y = layer), into the
+// group's workspace.  8 values per thread and step.  A value that f16 cannot hold (|q| >= 65520
+// rounds to infinity) sets DEVERR_RANGE, as the conversion inside the attention kernel does.
+struct QConvert {
+  const uint4* src[4];
+  uint4* dst[4];
+};
+__global__ void __launch_bounds__(256) q_to_f16_kernel(const __grid_constant__ QConvert qc, int64_t n_chunks, int* status) {
+  grid_dependency_sync();
+  const uint4* __restrict__ q = qc.src[blockIdx.y];
+  uint4* __restrict__ q16 = qc.dst[blockIdx.y];
+  bool out_of_range = false;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n_chunks;
+       i += static_cast<int64_t>(gridDim.x) * 256) {
+    const uint4 raw = q[i];
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xFFFF0000u);
+      out_of_range |= fmaxf(fabsf(lo), fabsf(hi)) >= 65520.f;
+      o[j] = pack_pair(lo, hi, true);
+    }
+    q16[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (out_of_range) atomicOr(status, DEVERR_RANGE);
 }
 
 // Combine split-KV partials: one CTA of 128 threads per (row, head), 4 dims per thread.  Equal

@@ -271,10 +271,13 @@ def test_decode_draft_step_reuses_the_handle():
                 assert np.max(np.abs(ls[row] - ref_lse)) <= 2e-3
 
 
-def test_paged_attention_query_values_within_and_beyond_f16_range():
+@pytest.mark.parametrize("k", [128, 2048])
+def test_paged_attention_query_values_within_and_beyond_f16_range(k):
     """Attention over an e4m3 cache runs its products on f16 operands: query values up to the f16
-    range give the oracle's result; a value beyond it is reported as DSA_ERR_RANGE."""
-    spec = DecodeSpec("q", batch=3, ctx_lo=200, ctx_hi=3000, rows_per_seq=2, k=128, n_layers=1, seed=13)
+    range give the oracle's result; a value beyond it is reported as DSA_ERR_RANGE.  k = 128: the
+    attention kernel converts the rows; k = 2048: 6 rows cut over 16 CTAs each, so the group
+    converts them ahead of the attention."""
+    spec = DecodeSpec("q", batch=3, ctx_lo=200, ctx_hi=3000, rows_per_seq=2, k=k, n_layers=1, seed=13)
     inp = make_decode(spec)
     Qb = O.bf16_to_f64(inp["Q"][0]).copy()
     Qb[:, 0, :4] = [20000.0, -20000.0, 12288.0, -30720.0]      # large, still finite in f16
