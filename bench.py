@@ -42,10 +42,10 @@ SUB_WORKLOADS = ["tiny_prefill", "prefill_32k", "decode_b32_mtp4", "decode_b32_d
 ALL_WORKLOADS = ["tiny_prefill", "prefill_32k", "prefill_128k_fp8", "decode_b32_mtp4", "decode_b32_d0",
                  "decode_b32_mtp4_verify", "decode_1m_mtp5"]
 
-# sparse_mla_kernel<bf16>, L=8,192 prefill launch (8,192 query rows): ncu measured 672.9 MB read
-# + 505.9 MB written = 143,893 B per query row (queries 73,728 B in, outputs 65,536 B out, the
+# sparse_mla_kernel<bf16>, L=8,192 prefill launch (8,192 query rows): ncu measured 672.8 MB read
+# + 505.5 MB written = 143,832 B per query row (queries 73,728 B in, outputs 65,536 B out, the
 # rest index rows and the latent rows' first touch).
-MLA_DRAM_BYTES_PER_ROW_BF16 = (672.903936e6 + 505.879296e6) / 8192
+MLA_DRAM_BYTES_PER_ROW_BF16 = (672.825600e6 + 505.489152e6) / 8192
 
 
 def parse(argv=None):
